@@ -1,0 +1,229 @@
+/*
+ * pkv.h -- C ABI of libpkv.so: paged KV-cache decode attention for NVIDIA
+ * B200 (sm_100a), plus the host-side block allocator that manages the pages.
+ *
+ * Sources for what each call computes (web pages, cited by title + section):
+ *   [KVB] "LLM Inference: KV Cache, Batching & Scheduling" (cariara.com),
+ *         sections "The KV cache" and "PagedAttention and vLLM".
+ *   [ENG] "LLM Inference Engineering: Overcoming the KV-Cache Bottleneck and
+ *         Maximizing Production Throughput" -- wpnews.pro summary, section
+ *         "2. The Architectural Solution: Virtual Memory and PagedAttention";
+ *         adilsher.pro post, section "The Elegant Fix: Paged Attention".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *   B  = number of sequences, Hq / Hkv = query / KV heads, G = Hq / Hkv,
+ *   D  = head_dim (64 or 128), bs = block_size (a multiple of 16), NB = pool
+ *   blocks, MB = max blocks per sequence (row length of the block table).
+ *
+ *   KV pool layout: k_cache and v_cache are two separate device arrays of
+ *   shape [NB][Hkv][bs][D] (16-bit floats), indexed by the same physical block
+ *   id.  The (block, kv-head) tile of bs*D elements is contiguous.  Position p
+ *   of a sequence lives in block block_tables[seq][p / bs], row p % bs.
+ *   A flat "slot" is block * bs + row.
+ *
+ *   Query head h attends with KV head h / G (contiguous query-head groups
+ *   share one KV head -- the GQA layout of [KVB] "The KV cache").
+ *
+ *   context_lens[s] is the sequence length AFTER this step's append: the
+ *   new token sits at position context_lens[s] - 1 and attention covers
+ *   positions 0 .. context_lens[s] - 1 inclusive.  A length of 0 produces an
+ *   all-zero output row.
+ *
+ * Ownership: the caller owns every device buffer (caches, q, out, tables,
+ * lengths, workspace).  The library never allocates or frees device memory
+ * in these calls; it owns only the allocator's host state.
+ *
+ * Errors: every call validates shapes, dtypes and alignment on the host and
+ * returns PKV_ERR_INVALID without launching anything.  Launches are
+ * asynchronous on the caller's stream; a launch failure returns PKV_ERR_CUDA.
+ * Device-side checks (a slot, table entry or length out of range) never trap:
+ * the kernel skips the access, records the fault in a device word and keeps
+ * going; pkv_get_last_error() reports it.  No call aborts the process.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID = -1,      /* bad argument; nothing was launched or changed      */
+    PKV_ERR_OOM = -2,          /* allocator: not enough free blocks; nothing changed */
+    PKV_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed               */
+    PKV_ERR_SHARED_WRITE = -4, /* allocator: the target block is shared (refcount>1) */
+    PKV_ERR_DEVICE_CHECK = -5, /* a kernel found an index out of range and skipped it */
+    PKV_ERR_TIMEOUT = -6       /* a kernel's bounded wait ran out and it returned early */
+} pkv_status;
+
+typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* One KV pool: caller-owned device pointer plus its shape [NB][Hkv][bs][D].
+ * data must be 16-byte aligned (TMA tiles are read straight from it). */
+typedef struct pkv_cache {
+    void *data;
+    pkv_dtype dtype;
+    int64_t num_blocks;
+    int64_t block_size;
+    int64_t num_kv_heads;
+    int64_t head_dim;
+} pkv_cache;
+
+/* A cudaStream_t without including CUDA headers (same underlying type). */
+struct CUstream_st;
+typedef struct CUstream_st *pkv_stream;
+
+/* --------------------------------------------------------------------------
+ * pkv_append -- store this step's new K and V of every token in its slot.
+ * [KVB] "The KV cache": the cache keeps K and V of every past position and
+ * appends the new token's K and V each step.
+ *
+ *   k_new, v_new   device [T][Hkv][D], same dtype and Hkv/D as the caches
+ *   slot_mapping   device int64 [T]; slot = block * bs + row; slot < 0 means
+ *                  "padding token, write nothing"
+ *   num_tokens     T >= 0 (T == 0 is a no-op)
+ *
+ * Bitwise copy: cache[slot / bs][h][slot % bs][:] = new[t][h][:] for all h.
+ * A slot with block >= NB is skipped and flagged (PKV_ERR_DEVICE_CHECK).
+ * Two tokens mapped to the same slot race (last writer unspecified).
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_append(const void *k_new, const void *v_new,
+                      const int64_t *slot_mapping, int64_t num_tokens,
+                      pkv_cache k_cache, pkv_cache v_cache, pkv_stream stream);
+
+/* --------------------------------------------------------------------------
+ * pkv_decode_attention -- one decode step of attention over the paged cache.
+ * [KVB] "The KV cache": attention needs the keys and values of all prior
+ * positions; decode generates one token at a time.  [KVB] "PagedAttention and
+ * vLLM" / [ENG]: K/V live in fixed-size blocks reached through a per-sequence
+ * logical -> physical block table; blocks need not be contiguous and may be
+ * shared between sequences (a common prefix).
+ *
+ *   out[s][h][:] = sum_p softmax_p(scale * q[s][h] . K[s][p]) * V[s][p]
+ *                  over p in [0, context_lens[s]), K/V of KV head h / G.
+ *
+ *   q              device [B][Hq][D], dtype of the caches
+ *   block_tables   device int32 [B][MB]; only the first
+ *                  ceil(context_lens[s] / bs) entries of row s are read
+ *   context_lens   device int32 [B], 0 <= len <= MB * bs
+ *   scale          softmax scale (usually 1/sqrt(D)), applied in fp32
+ *   out            device [B][Hq][D], dtype of q (round-to-nearest-even)
+ *   workspace      device scratch for split-context partial results, or NULL
+ *   partition_tokens
+ *       PKV_PARTITION_NONE (-1): one pass over each whole context; no
+ *                  workspace used.
+ *       PKV_PARTITION_AUTO (0): the library splits the total work evenly
+ *                  across the GPU (work-balanced partitions, merged by
+ *                  log-sum-exp); needs workspace >= the size reported by
+ *                  pkv_decode_workspace_bytes(..., 0).  With workspace NULL it
+ *                  falls back to PKV_PARTITION_NONE.
+ *       P > 0 (a multiple of 16): split every context into P-token
+ *                  partitions [jP, (j+1)P), computed independently and merged
+ *                  by log-sum-exp in a second kernel; workspace holds fp32
+ *                  partials [B][Hq][S][D] and their max / sum [B][Hq][S],
+ *                  S = ceil(MB * bs / P).
+ *
+ * Accumulation is fp32 throughout; exp via exp2 with scale*log2(e) folded in.
+ * Results do not depend on which physical blocks hold the data: the order of
+ * every reduction is fixed by logical position only.
+ * Limits: D in {64, 128}; bs a multiple of 16; Hq % Hkv == 0.
+ * ------------------------------------------------------------------------ */
+#define PKV_PARTITION_NONE (-1)
+#define PKV_PARTITION_AUTO 0
+
+pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_heads,
+                                pkv_cache k_cache, pkv_cache v_cache,
+                                const int32_t *block_tables, int64_t max_blocks_per_seq,
+                                const int32_t *context_lens, float scale, void *out,
+                                void *workspace, size_t workspace_bytes,
+                                int32_t partition_tokens, pkv_stream stream);
+
+/* Bytes of workspace pkv_decode_attention needs for this shape and
+ * partition_tokens on the CURRENT device (AUTO depends on its SM count).
+ * max_context_len is the largest context any sequence may have (MB * bs).
+ * Returns 0 for PKV_PARTITION_NONE and for invalid arguments. */
+size_t pkv_decode_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                  int64_t head_dim, int64_t max_context_len,
+                                  int32_t partition_tokens);
+
+/* --------------------------------------------------------------------------
+ * Host block allocator.  [KVB] "PagedAttention and vLLM": pages are
+ * allocated on demand and a finished request's pages return to the pool at
+ * once.  [ENG]: a memory manager maps logical blocks to physical blocks; two
+ * requests with the same prompt prefix share pages instead of duplicating.
+ *
+ * One handle manages one pool of num_blocks physical blocks (ids 0..NB-1)
+ * and any number of sequences.  Free blocks sit on a LIFO free list; every
+ * block carries a reference count (0 = free).  Not thread-safe: the caller
+ * serialises calls on one handle.  All calls are host-only.
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_alloc_create(int32_t num_blocks, int32_t block_size, void **handle);
+void pkv_alloc_destroy(void *handle);
+
+/* Pop a free block (refcount 0 -> 1).  PKV_ERR_OOM when none is free. */
+pkv_status pkv_block_alloc(void *h, int32_t *block_out);
+/* refcount += 1 on an allocated block (sharing it once more). */
+pkv_status pkv_block_incref(void *h, int32_t block);
+/* refcount -= 1; at 0 the block returns to the free list at once.
+ * PKV_ERR_INVALID for a free block (double free). */
+pkv_status pkv_block_decref(void *h, int32_t block);
+int32_t pkv_num_free(void *h);
+/* Reference count of a block, or -1 for an invalid id. */
+int32_t pkv_refcount(void *h, int32_t block);
+
+/* A new, empty sequence (context length 0, no blocks). */
+pkv_status pkv_seq_create(void *h, int32_t *seq_out);
+/* A new sequence that shares the parent's first num_full_blocks blocks
+ * (each gets one more reference) and starts with context length
+ * num_full_blocks * bs.  num_full_blocks * bs must not exceed the parent's
+ * length.  Only whole blocks are shared, so the child's next append opens a
+ * private block. */
+pkv_status pkv_seq_fork(void *h, int32_t parent, int32_t num_full_blocks, int32_t *child_out);
+/* Reserve the slot for the sequence's next token and return it
+ * (block * bs + row); the context length grows by one.  Opens a new block
+ * when the length is a multiple of bs (PKV_ERR_OOM if none is free).
+ * PKV_ERR_SHARED_WRITE if the token would land in a shared block.  On any
+ * error nothing changes. */
+pkv_status pkv_seq_append_slot(void *h, int32_t seq, int64_t *slot_out);
+/* pkv_seq_append_slot for n sequences at once, all or nothing: on an error
+ * (including OOM for the batch as a whole) no sequence changes. */
+pkv_status pkv_seq_append_slots(void *h, const int32_t *seqs, int32_t n, int64_t *slots_out);
+/* Drop the sequence: every block loses one reference; blocks reaching 0
+ * return to the free list.  The id may be reused by a later create/fork. */
+pkv_status pkv_seq_free(void *h, int32_t seq);
+/* Copy the sequence's block ids (logical order) to dst[0 .. min(n, cap)). */
+pkv_status pkv_seq_block_table(void *h, int32_t seq, int32_t *dst, int32_t cap, int32_t *n_out);
+/* Current context length of the sequence, or -1 for an invalid id. */
+int64_t pkv_seq_context_len(void *h, int32_t seq);
+/* Fill a batch block table dst[n][cap] (rows padded with -1) and
+ * context_lens[n] for the given sequences, ready to copy to the device. */
+pkv_status pkv_batch_tables(void *h, const int32_t *seqs, int32_t n, int32_t *dst,
+                            int32_t cap, int32_t *context_lens);
+
+/* Testing hook for the kernels' bounded waits (no counterpart on the pages).
+ * With enable != 0, decode launches made afterwards by this process issue no
+ * tile copies, so every wait for a tile runs out after wait_limit_ns (clamped
+ * to [1 ms, 2 s]); the kernel records the time-out and returns, and the CUDA
+ * context stays usable.  pkv_get_last_error() then reports PKV_ERR_TIMEOUT.
+ * enable == 0 restores normal operation (2 s limit).  Host-side setting only;
+ * nothing faults, traps or hangs. */
+pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns);
+
+/* Human-readable name of a status code (static storage). */
+const char *pkv_status_string(pkv_status s);
+/* Sticky error of the device checks, read and cleared.  Synchronises the
+ * current device.  PKV_ERR_TIMEOUT if a kernel's bounded wait ran out,
+ * PKV_ERR_DEVICE_CHECK if a kernel skipped an out-of-range access since the
+ * last call, PKV_ERR_CUDA on a pending CUDA error, else PKV_OK. */
+pkv_status pkv_get_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

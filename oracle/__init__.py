@@ -58,6 +58,8 @@ def _bind(lib):
         vp, i64, vp]
     lib.oracle_lse_merge.restype = ctypes.c_int
     lib.oracle_lse_merge.argtypes = [i64, vp, vp, vp, i64, vp]
+    lib.oracle_mark_slots.restype = ctypes.c_int
+    lib.oracle_mark_slots.argtypes = [vp, i64, i64, vp, i64, i64, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
     del i32
@@ -190,6 +192,18 @@ def lse_merge(m, l, o, lib=None) -> np.ndarray:
     out = np.zeros(d)
     lib.oracle_lse_merge(n, _p(m), _p(l), _p(o), d, _p(out))
     return out
+
+
+def slot_mask(block_tables, lens, block_size: int, num_blocks: int, lib=None) -> np.ndarray:
+    """bool [num_blocks * block_size]: True where a slot holds a position < lens[s] of some sequence."""
+    lib = lib or load()
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ln = np.ascontiguousarray(lens, dtype=np.int32)
+    mask = np.zeros(num_blocks * block_size, dtype=np.uint8)
+    rc = lib.oracle_mark_slots(_p(bt), bt.shape[0], bt.shape[1], _p(ln), block_size, num_blocks, _p(mask))
+    if rc != 0:
+        raise ValueError("oracle_mark_slots: table entry out of range")
+    return mask.astype(bool)
 
 
 def num_threads(lib=None) -> int:

@@ -324,3 +324,24 @@ void oracle_set_num_threads(int n)
     (void)n;
 #endif
 }
+
+/*
+ * Mark every slot (block * bs + row) that holds a position p < lens[s] of some
+ * sequence s: mask[slot] = 1.  Used by tests to poison every other slot.
+ * Returns -1 if a needed table entry is outside [0, num_blocks).
+ */
+int oracle_mark_slots(const int32_t *block_tables, int64_t num_seqs,
+                      int64_t max_blocks_per_seq, const int32_t *lens,
+                      int64_t block_size, int64_t num_blocks, uint8_t *mask)
+{
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        const int32_t *row = block_tables + s * max_blocks_per_seq;
+        for (int64_t p = 0; p < lens[s]; ++p) {
+            int64_t b = row[p / block_size];
+            if (b < 0 || b >= num_blocks)
+                return -1;
+            mask[b * block_size + p % block_size] = 1;
+        }
+    }
+    return 0;
+}

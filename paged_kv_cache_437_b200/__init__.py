@@ -1,0 +1,312 @@
+"""Python binding of ``libpkv.so`` -- paged KV-cache decode attention on B200.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels (sm_100a) or its C++ host allocator.  There is no fallback: if the
+shared library is missing, importing this package raises ``ImportError``.
+Build it with ``python paged_kv_cache_437_b200/build.py``.
+
+Names follow the C ABI in ``include/pkv.h``.  Device buffers are passed as
+torch CUDA tensors (torch is used for device memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+PKV_OK = 0
+PKV_ERR_INVALID = -1
+PKV_ERR_OOM = -2
+PKV_ERR_CUDA = -3
+PKV_ERR_SHARED_WRITE = -4
+PKV_ERR_DEVICE_CHECK = -5
+PKV_ERR_TIMEOUT = -6
+
+PKV_F16 = 0
+PKV_BF16 = 1
+
+PKV_PARTITION_NONE = -1
+PKV_PARTITION_AUTO = 0
+
+_c_i32, _c_i64, _c_vp, _c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+
+
+class pkv_cache(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int), ("num_blocks", ctypes.c_int64),
+                ("block_size", ctypes.c_int64), ("num_kv_heads", ctypes.c_int64),
+                ("head_dim", ctypes.c_int64)]
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {pkv_status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_437_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "pkv_append": (ctypes.c_int, [_c_vp, _c_vp, _c_vp, _c_i64, pkv_cache, pkv_cache, _c_vp]),
+        "pkv_decode_attention": (ctypes.c_int, [_c_vp, _c_i64, _c_i64, pkv_cache, pkv_cache, _c_vp, _c_i64,
+                                                _c_vp, ctypes.c_float, _c_vp, _c_vp, _c_sz, _c_i32, _c_vp]),
+        "pkv_decode_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i32]),
+        "pkv_alloc_create": (ctypes.c_int, [_c_i32, _c_i32, ctypes.POINTER(_c_vp)]),
+        "pkv_alloc_destroy": (None, [_c_vp]),
+        "pkv_block_alloc": (ctypes.c_int, [_c_vp, ctypes.POINTER(_c_i32)]),
+        "pkv_block_incref": (ctypes.c_int, [_c_vp, _c_i32]),
+        "pkv_block_decref": (ctypes.c_int, [_c_vp, _c_i32]),
+        "pkv_num_free": (_c_i32, [_c_vp]),
+        "pkv_refcount": (_c_i32, [_c_vp, _c_i32]),
+        "pkv_seq_create": (ctypes.c_int, [_c_vp, ctypes.POINTER(_c_i32)]),
+        "pkv_seq_fork": (ctypes.c_int, [_c_vp, _c_i32, _c_i32, ctypes.POINTER(_c_i32)]),
+        "pkv_seq_append_slot": (ctypes.c_int, [_c_vp, _c_i32, ctypes.POINTER(_c_i64)]),
+        "pkv_seq_append_slots": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp]),
+        "pkv_seq_free": (ctypes.c_int, [_c_vp, _c_i32]),
+        "pkv_seq_block_table": (ctypes.c_int, [_c_vp, _c_i32, _c_vp, _c_i32, ctypes.POINTER(_c_i32)]),
+        "pkv_seq_context_len": (_c_i64, [_c_vp, _c_i32]),
+        "pkv_batch_tables": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_i32, _c_vp]),
+        "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "pkv_get_last_error": (ctypes.c_int, []),
+        "pkv_test_inject_wait_timeout": (ctypes.c_int, [_c_i32, _c_i64]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def pkv_status_string(status: int) -> str:
+    return lib.pkv_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != PKV_OK:
+        raise PkvError(status, what)
+
+
+# ------------------------------------------------------------------ device calls
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.float16:
+        return PKV_F16
+    if t.dtype == torch.bfloat16:
+        return PKV_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float16 or bfloat16")
+
+
+def _stream_ptr(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _require(t, name, ndim=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def cache_desc(cache) -> pkv_cache:
+    """Describe a [NB][Hkv][bs][D] fp16/bf16 CUDA tensor as a ``pkv_cache``."""
+    _require(cache, "cache", 4)
+    nb, hkv, bs, d = cache.shape
+    return pkv_cache(cache.data_ptr(), _dtype_code(cache), nb, bs, hkv, d)
+
+
+def pkv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """Write k_new/v_new [T][Hkv][D] into the caches at slot_mapping[T] (int64, <0 = skip)."""
+    import torch
+
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (slot_mapping, "slot_mapping")):
+        _require(t, n)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    if k_new.dtype != k_cache.dtype or v_new.dtype != v_cache.dtype:
+        raise TypeError("new K/V must have the caches' dtype")
+    if k_new.shape != v_new.shape or k_new.dim() != 3 or k_new.shape[0] != slot_mapping.numel() or \
+            k_new.shape[1] != k_cache.shape[1] or k_new.shape[2] != k_cache.shape[3]:
+        raise ValueError("k_new / v_new must be [T][Hkv][D] with T = len(slot_mapping)")
+    st = lib.pkv_append(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(), slot_mapping.numel(),
+                        cache_desc(k_cache), cache_desc(v_cache), _stream_ptr(stream))
+    _check(st, "pkv_append")
+
+
+def pkv_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                               max_context_len: int, partition_tokens: int = PKV_PARTITION_AUTO) -> int:
+    return int(lib.pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              max_context_len, partition_tokens))
+
+
+def pkv_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                         workspace=None, partition_tokens: int = PKV_PARTITION_AUTO, stream=None) -> None:
+    """out[B][Hq][D] = paged decode attention of q[B][Hq][D] over the caches."""
+    import torch
+
+    for t, n in ((q, "q"), (out, "out"), (block_tables, "block_tables"), (context_lens, "context_lens")):
+        _require(t, n)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if q.dtype != k_cache.dtype or out.dtype != q.dtype:
+        raise TypeError("q, out and the caches must share one dtype")
+    if q.dim() != 3 or out.shape != q.shape or block_tables.dim() != 2 or \
+            block_tables.shape[0] != q.shape[0] or context_lens.numel() != q.shape[0]:
+        raise ValueError("shapes: q/out [B][Hq][D], block_tables [B][MB], context_lens [B]")
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        _require(workspace, "workspace")
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = lib.pkv_decode_attention(q.data_ptr(), q.shape[0], q.shape[1], cache_desc(k_cache),
+                                  cache_desc(v_cache), block_tables.data_ptr(), block_tables.shape[1],
+                                  context_lens.data_ptr(), float(scale), out.data_ptr(), ws_ptr or None,
+                                  ws_bytes, int(partition_tokens), _stream_ptr(stream))
+    _check(st, "pkv_decode_attention")
+
+
+def pkv_test_inject_wait_timeout(enable: bool, wait_limit_ns: int = 50_000_000) -> None:
+    _check(lib.pkv_test_inject_wait_timeout(1 if enable else 0, int(wait_limit_ns)),
+           "pkv_test_inject_wait_timeout")
+
+
+def pkv_get_last_error() -> int:
+    """Read-and-clear the device check word (synchronises the device)."""
+    return int(lib.pkv_get_last_error())
+
+
+# ------------------------------------------------------------------ host allocator
+
+def pkv_alloc_create(num_blocks: int, block_size: int):
+    h = ctypes.c_void_p()
+    _check(lib.pkv_alloc_create(num_blocks, block_size, ctypes.byref(h)), "pkv_alloc_create")
+    return h
+
+
+def pkv_alloc_destroy(h) -> None:
+    lib.pkv_alloc_destroy(h)
+
+
+def pkv_block_alloc(h) -> int:
+    b = ctypes.c_int32()
+    _check(lib.pkv_block_alloc(h, ctypes.byref(b)), "pkv_block_alloc")
+    return b.value
+
+
+def pkv_block_incref(h, block: int) -> None:
+    _check(lib.pkv_block_incref(h, block), "pkv_block_incref")
+
+
+def pkv_block_decref(h, block: int) -> None:
+    _check(lib.pkv_block_decref(h, block), "pkv_block_decref")
+
+
+def pkv_num_free(h) -> int:
+    return int(lib.pkv_num_free(h))
+
+
+def pkv_refcount(h, block: int) -> int:
+    return int(lib.pkv_refcount(h, block))
+
+
+def pkv_seq_create(h) -> int:
+    s = ctypes.c_int32()
+    _check(lib.pkv_seq_create(h, ctypes.byref(s)), "pkv_seq_create")
+    return s.value
+
+
+def pkv_seq_fork(h, parent: int, num_full_blocks: int) -> int:
+    s = ctypes.c_int32()
+    _check(lib.pkv_seq_fork(h, parent, num_full_blocks, ctypes.byref(s)), "pkv_seq_fork")
+    return s.value
+
+
+def pkv_seq_append_slot(h, seq: int) -> int:
+    slot = ctypes.c_int64()
+    _check(lib.pkv_seq_append_slot(h, seq, ctypes.byref(slot)), "pkv_seq_append_slot")
+    return slot.value
+
+
+def pkv_seq_append_slots(h, seqs):
+    """Slots (numpy int64) for one new token of each sequence; all or nothing."""
+    import numpy as np
+
+    s = np.ascontiguousarray(seqs, dtype=np.int32)
+    out = np.empty(len(s), dtype=np.int64)
+    _check(lib.pkv_seq_append_slots(h, s.ctypes.data, len(s), out.ctypes.data), "pkv_seq_append_slots")
+    return out
+
+
+def pkv_seq_free(h, seq: int) -> None:
+    _check(lib.pkv_seq_free(h, seq), "pkv_seq_free")
+
+
+def pkv_seq_block_table(h, seq: int):
+    import numpy as np
+
+    n = ctypes.c_int32()
+    _check(lib.pkv_seq_block_table(h, seq, None, 0, ctypes.byref(n)), "pkv_seq_block_table")
+    out = np.empty(n.value, dtype=np.int32)
+    _check(lib.pkv_seq_block_table(h, seq, out.ctypes.data, n.value, ctypes.byref(n)), "pkv_seq_block_table")
+    return out
+
+
+def pkv_seq_context_len(h, seq: int) -> int:
+    return int(lib.pkv_seq_context_len(h, seq))
+
+
+def pkv_batch_tables(h, seqs, cap: int):
+    """(block_tables [n][cap] int32 padded with -1, context_lens [n] int32) for a batch."""
+    import numpy as np
+
+    s = np.ascontiguousarray(seqs, dtype=np.int32)
+    tables = np.empty((len(s), cap), dtype=np.int32)
+    lens = np.empty(len(s), dtype=np.int32)
+    _check(lib.pkv_batch_tables(h, s.ctypes.data, len(s), tables.ctypes.data, cap, lens.ctypes.data),
+           "pkv_batch_tables")
+    return tables, lens
+
+
+class BlockAllocator:
+    """Owning wrapper of one allocator handle."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        self.handle = pkv_alloc_create(num_blocks, block_size)
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def close(self):
+        if self.handle:
+            pkv_alloc_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    alloc = lambda self: pkv_block_alloc(self.handle)
+    incref = lambda self, b: pkv_block_incref(self.handle, b)
+    decref = lambda self, b: pkv_block_decref(self.handle, b)
+    num_free = lambda self: pkv_num_free(self.handle)
+    refcount = lambda self, b: pkv_refcount(self.handle, b)
+    seq_create = lambda self: pkv_seq_create(self.handle)
+    seq_fork = lambda self, p, n: pkv_seq_fork(self.handle, p, n)
+    append_slot = lambda self, s: pkv_seq_append_slot(self.handle, s)
+    append_slots = lambda self, seqs: pkv_seq_append_slots(self.handle, seqs)
+    seq_free = lambda self, s: pkv_seq_free(self.handle, s)
+    block_table = lambda self, s: pkv_seq_block_table(self.handle, s)
+    context_len = lambda self, s: pkv_seq_context_len(self.handle, s)
+    batch_tables = lambda self, seqs, cap: pkv_batch_tables(self.handle, seqs, cap)

@@ -1,0 +1,442 @@
+// C ABI of the device calls: argument validation, TMA tensor maps, launch
+// planning and the split-context workspace layout.  Every kernel lives in
+// decode.cuh (one translation unit so that the device error word is shared).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "decode.cuh"
+#include "pkv.h"
+
+namespace pkv {
+
+__device__ unsigned g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxSmemPerCta = 226 * 1024;  // 227 KB opt-in limit minus static smem
+
+// testing hook state (pkv_test_inject_wait_timeout)
+int g_inject_no_issue = 0;
+uint64_t g_wait_limit_ns = kWaitLimitNs;
+
+int env_int(const char *name, int dflt) {
+    const char *v = std::getenv(name);
+    if (!v || !*v)
+        return dflt;
+    return std::atoi(v);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool cache_ok(const pkv_cache &c) {
+    return c.data && aligned16(c.data) && (c.dtype == PKV_F16 || c.dtype == PKV_BF16) &&
+           c.num_blocks > 0 && c.block_size > 0 && c.num_kv_heads > 0 && c.head_dim > 0;
+}
+
+bool same_shape(const pkv_cache &a, const pkv_cache &b) {
+    return a.dtype == b.dtype && a.num_blocks == b.num_blocks && a.block_size == b.block_size &&
+           a.num_kv_heads == b.num_kv_heads && a.head_dim == b.head_dim;
+}
+
+unsigned *error_word() {
+    static unsigned *ptr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    if (!ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess)
+            return nullptr;
+        ptr[dev] = static_cast<unsigned *>(p);
+    }
+    return ptr[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// The pool viewed as a 2-D tensor: rows = NB * Hkv * bs, columns = D; one TMA
+// box = 16 rows x 64 columns (128 bytes per row), 128-byte swizzle.
+bool make_pool_map(CUtensorMap *map, const pkv_cache &c) {
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)c.head_dim,
+                          (cuuint64_t)(c.num_blocks * c.num_kv_heads * c.block_size)};
+    cuuint64_t strides[1] = {(cuuint64_t)c.head_dim * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)kTileTokens};
+    cuuint32_t estr[2] = {1, 1};
+    CUtensorMapDataType dt =
+        c.dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(map, dt, 2, c.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct Plan {
+    int mode = kModeDirect;
+    int warps = 4;
+    int stages = 3;
+    int ctas = 0;
+    int total_warps = 0;
+    int max_total_warps = 0;  // warps of the largest grid this shape may launch
+    int part_tiles = 0;
+    int S = 0;
+    int smem = 0;
+    int Hkv = 0, G = 0, n_hg = 0, npairs = 0;
+};
+
+using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
+
+DecodeKernel pick_decode(int D, bool bf16, bool two) {
+#define PKV_PICK(DD, BB, TT) \
+    if (D == DD && bf16 == BB && two == TT) return paged_decode_kernel<DD, BB, TT>;
+    PKV_PICK(64, false, false)
+    PKV_PICK(64, false, true)
+    PKV_PICK(64, true, false)
+    PKV_PICK(64, true, true)
+    PKV_PICK(128, false, false)
+    PKV_PICK(128, false, true)
+    PKV_PICK(128, true, false)
+    PKV_PICK(128, true, true)
+#undef PKV_PICK
+    return nullptr;
+}
+
+int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Decide schedule, CTA shape and grid.  PKV_ERR_INVALID if the shape cannot
+// be run (shared memory), PKV_ERR_CUDA if the device cannot be queried.
+pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
+               int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch) {
+    p.Hkv = (int)Hkv;
+    p.G = (int)(Hq / Hkv);
+    p.n_hg = (p.G + kMaxRows - 1) / kMaxRows;
+    p.npairs = (int)Hkv * p.n_hg;
+    p.warps = env_int("PKV_WARPS", 4);
+    p.stages = env_int("PKV_STAGES", D == 64 ? 6 : 3);
+    if (p.warps < 1 || p.warps > 8)
+        p.warps = 4;
+    if (p.stages < 2 || p.stages > 16)
+        p.stages = 3;
+    if (partition_tokens > 0) {
+        p.mode = kModePartition;
+        p.part_tiles = partition_tokens / kTileTokens;
+        p.S = (int)ceil_div64(max_ctx, partition_tokens);
+        if (p.S < 1)
+            p.S = 1;
+    } else if (partition_tokens == PKV_PARTITION_AUTO && have_workspace) {
+        p.mode = kModeBalanced;
+    } else {
+        p.mode = kModeDirect;
+    }
+    const bool need_prefix = p.mode != kModeDirect;
+    // the on-chip schedule keeps per-sequence tile counts in int32
+    if (need_prefix && B * ceil_div64(max_ctx, kTileTokens) * p.npairs >= (int64_t(1) << 31))
+        return PKV_ERR_INVALID;
+    for (;;) {
+        SmemLayout L = decode_smem_layout((int)B, p.warps, p.stages, (int)D, need_prefix);
+        p.smem = L.total;
+        if (p.smem <= kMaxSmemPerCta)
+            break;
+        if (p.stages > 2)
+            --p.stages;
+        else if (p.warps > 1)
+            --p.warps;
+        else
+            return PKV_ERR_INVALID;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int per_sm = 1;
+    DecodeKernel k = pick_decode((int)D, bf16, p.G > 8);
+    if (!k)
+        return PKV_ERR_INVALID;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, p.warps * 32, p.smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t max_ctas = (int64_t)sms * per_sm;
+    p.max_total_warps = (int)(max_ctas * p.warps);
+    int64_t want = max_ctas;
+    if (for_launch) {
+        const int64_t tiles_upper = ceil_div64(max_ctx, kTileTokens);
+        int64_t units;
+        if (p.mode == kModeDirect)
+            units = B * p.npairs;
+        else if (p.mode == kModePartition)
+            units = B * p.npairs * p.S;
+        else
+            units = ceil_div64(B * p.npairs * tiles_upper, 4);  // >= ~4 tiles per warp
+        want = std::min<int64_t>(max_ctas, std::max<int64_t>(1, ceil_div64(units, p.warps)));
+    }
+    p.ctas = (int)want;
+    p.total_warps = p.ctas * p.warps;
+    return PKV_OK;
+}
+
+// Workspace layout.
+//  partition: part_o [B][Hq][S][D] f32 | part_m [B][Hq][S] f32 | part_l [B][Hq][S] f32
+//  balanced:  prefix [B+1] i32 (256-aligned) | part_m [2W][16] | part_l [2W][16] | part_o [2W][16][D]
+//             with W = the largest warp count a launch may use.
+struct WsLayout {
+    size_t prefix = 0, m = 0, l = 0, o = 0, total = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const Plan &p, int64_t B, int64_t Hq, int64_t D, int64_t max_warps) {
+    WsLayout w;
+    if (p.mode == kModePartition) {
+        const size_t rows = (size_t)B * Hq * p.S;
+        w.o = 0;
+        w.m = align256(rows * D * 4);
+        w.l = align256(w.m + rows * 4);
+        w.total = align256(w.l + rows * 4);
+    } else if (p.mode == kModeBalanced) {
+        const size_t slots = (size_t)2 * max_warps;
+        w.prefix = 0;
+        w.m = align256((size_t)(B + 1) * 4);
+        w.l = align256(w.m + slots * kMaxRows * 4);
+        w.o = align256(w.l + slots * kMaxRows * 4);
+        w.total = align256(w.o + slots * kMaxRows * D * 4);
+    }
+    return w;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+pkv_status pkv_append(const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                      int64_t num_tokens, pkv_cache k_cache, pkv_cache v_cache, pkv_stream stream) {
+    if (num_tokens < 0)
+        return PKV_ERR_INVALID;
+    if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
+        return PKV_ERR_INVALID;
+    if (k_cache.head_dim % 8 != 0)
+        return PKV_ERR_INVALID;
+    if (num_tokens == 0)
+        return PKV_OK;
+    if (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID;
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+    const int chunks = (int)(k_cache.head_dim / 8);
+    const int64_t total = num_tokens * k_cache.num_kv_heads * chunks;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > 148 * 32)
+        blocks = 148 * 32;
+    append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping,
+        num_tokens, (int)k_cache.num_kv_heads, chunks, (int)k_cache.block_size,
+        k_cache.num_blocks, static_cast<uint4 *>(k_cache.data), static_cast<uint4 *>(v_cache.data),
+        err);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+size_t pkv_decode_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                  int64_t head_dim, int64_t max_context_len,
+                                  int32_t partition_tokens) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+        (head_dim != 64 && head_dim != 128) || max_context_len < 0)
+        return 0;
+    if (partition_tokens == PKV_PARTITION_NONE)
+        return 0;
+    if (partition_tokens < 0 || partition_tokens % kTileTokens)
+        return 0;
+    Plan p;
+    if (make_plan(p, num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                  partition_tokens, true, false, false) != PKV_OK)
+        return 0;
+    return ws_layout(p, num_seqs, num_q_heads, head_dim, p.max_total_warps).total;
+}
+
+pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_heads,
+                                pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+                                int64_t max_blocks_per_seq, const int32_t *context_lens,
+                                float scale, void *out, void *workspace, size_t workspace_bytes,
+                                int32_t partition_tokens, pkv_stream stream) {
+    if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0)
+        return PKV_ERR_INVALID;
+    if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
+        return PKV_ERR_INVALID;
+    const int64_t Hkv = k_cache.num_kv_heads, D = k_cache.head_dim, bs = k_cache.block_size;
+    if (num_q_heads % Hkv != 0 || (D != 64 && D != 128) || bs % kTileTokens != 0)
+        return PKV_ERR_INVALID;
+    if (!std::isfinite(scale))
+        return PKV_ERR_INVALID;
+    if (partition_tokens < PKV_PARTITION_NONE ||
+        (partition_tokens > 0 && partition_tokens % kTileTokens != 0))
+        return PKV_ERR_INVALID;
+    // TMA coordinates are 32-bit; the row count of the pool view must fit
+    if (k_cache.num_blocks * Hkv * bs >= (int64_t(1) << 31))
+        return PKV_ERR_INVALID;
+    if (max_blocks_per_seq * bs >= (int64_t(1) << 30) || num_seqs >= (int64_t(1) << 24) ||
+        num_q_heads * D >= (int64_t(1) << 24))
+        return PKV_ERR_INVALID;
+    if (num_seqs == 0)
+        return PKV_OK;
+    if (!q || !out || !block_tables || !context_lens || !aligned16(q) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PKV_ERR_INVALID;
+    const bool bf16 = k_cache.dtype == PKV_BF16;
+    const int64_t max_ctx = max_blocks_per_seq * bs;
+    const bool have_ws = workspace != nullptr;
+    if (have_ws && !aligned16(workspace))
+        return PKV_ERR_INVALID;
+    if (partition_tokens > 0 && !have_ws)
+        return PKV_ERR_INVALID;
+
+    Plan p;
+    pkv_status ps = make_plan(p, num_seqs, num_q_heads, Hkv, D, max_ctx, partition_tokens, have_ws,
+                              bf16, true);
+    if (ps == PKV_ERR_INVALID && partition_tokens == PKV_PARTITION_AUTO) {
+        // AUTO with a batch too large for the on-chip schedule: one pass per unit
+        ps = make_plan(p, num_seqs, num_q_heads, Hkv, D, max_ctx, PKV_PARTITION_NONE, false, bf16, true);
+    }
+    if (ps != PKV_OK)
+        return ps;
+    WsLayout wl;
+    if (p.mode != kModeDirect) {
+        wl = ws_layout(p, num_seqs, num_q_heads, D, p.max_total_warps);
+        if (workspace_bytes < wl.total)
+            return PKV_ERR_INVALID;
+    }
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+
+    CUtensorMap tmK, tmV;
+    if (!make_pool_map(&tmK, k_cache) || !make_pool_map(&tmV, v_cache))
+        return PKV_ERR_CUDA;
+
+    DecodeArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.out = static_cast<uint16_t *>(out);
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.mb = max_blocks_per_seq;
+    a.nb = k_cache.num_blocks;
+    a.B = (int)num_seqs;
+    a.Hq = (int)num_q_heads;
+    a.Hkv = (int)Hkv;
+    a.G = p.G;
+    a.n_hg = p.n_hg;
+    a.npairs = p.npairs;
+    a.bs = (int)bs;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.mode = p.mode;
+    a.part_tiles = p.part_tiles;
+    a.S = p.S;
+    char *ws = static_cast<char *>(workspace);
+    a.part_o = have_ws ? reinterpret_cast<float *>(ws + wl.o) : nullptr;
+    a.part_m = have_ws ? reinterpret_cast<float *>(ws + wl.m) : nullptr;
+    a.part_l = have_ws ? reinterpret_cast<float *>(ws + wl.l) : nullptr;
+    a.prefix_out = have_ws ? reinterpret_cast<int32_t *>(ws + wl.prefix) : nullptr;
+    a.total_warps = p.total_warps;
+    a.stages = p.stages;
+    a.err = err;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.inject_no_issue = g_inject_no_issue;
+
+    DecodeKernel k = pick_decode((int)D, bf16, p.G > 8);
+    k<<<p.ctas, p.warps * 32, p.smem, (cudaStream_t)stream>>>(tmK, tmV, a);
+    if (cudaGetLastError() != cudaSuccess)
+        return PKV_ERR_CUDA;
+
+    const bool merge = (p.mode == kModeBalanced) || (p.mode == kModePartition && p.S > 1);
+    if (merge) {
+        MergeArgs m;
+        m.out = a.out;
+        m.context_lens = context_lens;
+        m.prefix = a.prefix_out;
+        m.part_o = a.part_o;
+        m.part_m = a.part_m;
+        m.part_l = a.part_l;
+        m.mb = max_blocks_per_seq;
+        m.B = a.B;
+        m.Hq = a.Hq;
+        m.G = a.G;
+        m.n_hg = a.n_hg;
+        m.npairs = a.npairs;
+        m.bs = a.bs;
+        m.D = (int)D;
+        m.mode = p.mode;
+        m.part_tiles = p.part_tiles;
+        m.S = p.S;
+        m.total_warps = p.total_warps;
+        m.err = err;
+        const int64_t grid = num_seqs * p.npairs;
+        if (bf16)
+            lse_merge_kernel<true><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(m);
+        else
+            lse_merge_kernel<false><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(m);
+        if (cudaGetLastError() != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_get_last_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return PKV_ERR_CUDA;
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    if (v != 0) {
+        const unsigned zero = 0;
+        cudaMemcpy(err, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        return (v & kErrTimeout) ? PKV_ERR_TIMEOUT : PKV_ERR_DEVICE_CHECK;
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns) {
+    if (enable) {
+        if (wait_limit_ns < 1000000)
+            wait_limit_ns = 1000000;
+        if (wait_limit_ns > (int64_t)kWaitLimitNs)
+            wait_limit_ns = (int64_t)kWaitLimitNs;
+        g_inject_no_issue = 1;
+        g_wait_limit_ns = (uint64_t)wait_limit_ns;
+    } else {
+        g_inject_no_issue = 0;
+        g_wait_limit_ns = kWaitLimitNs;
+    }
+    return PKV_OK;
+}
+
+}  // extern "C"

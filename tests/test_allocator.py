@@ -1,0 +1,187 @@
+"""Host block allocator (free list, refcounts, sequences), CPU only.
+
+Slot addresses are checked against the oracle's slot function and against
+brute-force enumeration of each sequence's blocks."""
+import numpy as np
+import pytest
+
+import oracle
+
+pkv = pytest.importorskip("paged_kv_cache_437_b200")
+
+
+def test_alloc_until_oom_and_return():
+    a = pkv.BlockAllocator(8, 16)
+    got = [a.alloc() for _ in range(8)]
+    assert sorted(got) == list(range(8))
+    assert a.num_free() == 0
+    with pytest.raises(pkv.PkvError) as e:
+        a.alloc()
+    assert e.value.status == pkv.PKV_ERR_OOM
+    for b in got:
+        assert a.refcount(b) == 1
+        a.decref(b)
+        assert a.refcount(b) == 0
+    assert a.num_free() == 8
+
+
+def test_refcounts_and_double_free():
+    a = pkv.BlockAllocator(4, 16)
+    b = a.alloc()
+    a.incref(b)
+    a.incref(b)
+    assert a.refcount(b) == 3
+    a.decref(b)
+    a.decref(b)
+    assert a.num_free() == 3
+    a.decref(b)
+    assert a.num_free() == 4 and a.refcount(b) == 0
+    with pytest.raises(pkv.PkvError) as e:
+        a.decref(b)
+    assert e.value.status == pkv.PKV_ERR_INVALID
+    with pytest.raises(pkv.PkvError):
+        a.incref(b)
+    assert a.refcount(-1) == -1 and a.refcount(4) == -1
+    with pytest.raises(pkv.PkvError):
+        a.decref(99)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_append_slots_match_oracle_and_bruteforce(orc, bs):
+    rng = np.random.default_rng(0)
+    a = pkv.BlockAllocator(64, bs)
+    seqs = [a.seq_create() for _ in range(3)]
+    lengths = [5, 40, 70]
+    slots = {s: [] for s in seqs}
+    for step in range(max(lengths)):
+        for s, n in zip(seqs, lengths):
+            if step < n:
+                slots[s].append(a.append_slot(s))
+    for s, n in zip(seqs, lengths):
+        table = a.block_table(s)
+        assert len(table) == -(-n // bs)
+        assert a.context_len(s) == n
+        enum = []
+        for blk in table:  # brute force: block by block, row by row
+            enum.extend(int(blk) * bs + r for r in range(bs))
+        assert slots[s] == enum[:n]
+        assert slots[s] == [oracle.slot_of(table, p, bs, lib=orc) for p in range(n)]
+    all_blocks = np.concatenate([a.block_table(s) for s in seqs])
+    assert len(set(all_blocks.tolist())) == len(all_blocks)  # no block owned twice
+    del rng
+
+
+def test_seq_free_returns_blocks_at_once():
+    a = pkv.BlockAllocator(10, 16)
+    s = a.seq_create()
+    for _ in range(33):
+        a.append_slot(s)
+    assert a.num_free() == 7
+    a.seq_free(s)
+    assert a.num_free() == 10
+    with pytest.raises(pkv.PkvError):
+        a.append_slot(s)
+    s2 = a.seq_create()       # id reuse is allowed
+    assert a.context_len(s2) == 0
+
+
+def test_fork_shares_full_prefix_blocks():
+    a = pkv.BlockAllocator(16, 16)
+    p = a.seq_create()
+    for _ in range(40):       # blocks: 16 + 16 + 8
+        a.append_slot(p)
+    parent_table = a.block_table(p)
+    c = a.seq_fork(p, 2)
+    assert list(a.block_table(c)) == list(parent_table[:2])
+    assert a.context_len(c) == 32
+    for b in parent_table[:2]:
+        assert a.refcount(int(b)) == 2
+    assert a.refcount(int(parent_table[2])) == 1
+    slot = a.append_slot(c)   # opens a private block
+    assert slot // 16 not in parent_table.tolist()
+    assert a.refcount(slot // 16) == 1
+    a.seq_free(p)
+    for b in parent_table[:2]:
+        assert a.refcount(int(b)) == 1
+    assert a.refcount(int(parent_table[2])) == 0
+    a.seq_free(c)
+    assert a.num_free() == 16
+
+
+def test_write_into_shared_block_is_refused_without_change():
+    a = pkv.BlockAllocator(8, 16)
+    p = a.seq_create()
+    for _ in range(20):
+        a.append_slot(p)
+    c = a.seq_fork(p, 1)
+    # make the parent's second block shared too, then try to write into it
+    b1 = int(a.block_table(p)[1])
+    a.incref(b1)
+    free_before = a.num_free()
+    with pytest.raises(pkv.PkvError) as e:
+        a.append_slot(p)
+    assert e.value.status == pkv.PKV_ERR_SHARED_WRITE
+    assert a.context_len(p) == 20 and a.num_free() == free_before
+    a.decref(b1)
+    a.append_slot(p)
+    assert a.context_len(p) == 21
+    del c
+
+
+def test_fork_argument_checks():
+    a = pkv.BlockAllocator(8, 16)
+    p = a.seq_create()
+    for _ in range(20):
+        a.append_slot(p)
+    with pytest.raises(pkv.PkvError):
+        a.seq_fork(p, 2)      # 32 > 20 tokens
+    with pytest.raises(pkv.PkvError):
+        a.seq_fork(p, -1)
+    with pytest.raises(pkv.PkvError):
+        a.seq_fork(77, 0)
+
+
+def test_batch_append_is_all_or_nothing():
+    a = pkv.BlockAllocator(3, 16)
+    s = [a.seq_create() for _ in range(3)]
+    a.append_slots(s)                      # 3 blocks used
+    assert a.num_free() == 0
+    for _ in range(15):
+        a.append_slots(s)                  # fills every block
+    before = [a.context_len(x) for x in s]
+    with pytest.raises(pkv.PkvError) as e:
+        a.append_slots(s)                  # needs 3 new blocks, none free
+    assert e.value.status == pkv.PKV_ERR_OOM
+    assert [a.context_len(x) for x in s] == before
+    with pytest.raises(pkv.PkvError) as e:
+        a.append_slots([s[0], s[0]])
+    assert e.value.status == pkv.PKV_ERR_INVALID
+
+
+def test_batch_tables():
+    a = pkv.BlockAllocator(32, 16)
+    s = [a.seq_create() for _ in range(3)]
+    for n, x in zip([1, 17, 40], s):
+        for _ in range(n):
+            a.append_slot(x)
+    tables, lens = a.batch_tables(s, 4)
+    assert lens.tolist() == [1, 17, 40]
+    for i, x in enumerate(s):
+        t = a.block_table(x)
+        assert tables[i, :len(t)].tolist() == t.tolist()
+        assert (tables[i, len(t):] == -1).all()
+    with pytest.raises(pkv.PkvError):
+        a.batch_tables(s, 2)               # row too short for 3 blocks
+
+
+def test_shuffled_free_list_via_public_api():
+    """Draining then returning blocks in a chosen order makes later pops come
+    out in the reverse of that order (LIFO), so a seeded permutation of the
+    pool can be reproduced through the allocator alone."""
+    a = pkv.BlockAllocator(20, 16)
+    got = [a.alloc() for _ in range(20)]
+    perm = np.random.default_rng(3).permutation(20)
+    for b in perm[::-1]:
+        a.decref(int(got[b]))
+    again = [a.alloc() for _ in range(20)]
+    assert again == [int(got[b]) for b in perm]
