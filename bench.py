@@ -1,0 +1,614 @@
+"""Benchmark one paged decode step (append + attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--partition P] [--flush-l2] [--impl reference]
+
+A step is the whole hot path on one batch: pkv_append of every sequence's new
+token, then pkv_decode_attention (decode kernel + log-sum-exp merge when the
+schedule splits contexts).  Inputs are synthetic and seeded (``workloads``),
+shaped like the pages' examples; the default workload is the 13B-shaped layer
+(32 sequences x 2048 context, 40/40 heads, D 128, block 16, fp16).
+
+Metric: achieved HBM GB/s of algorithmic bytes (KV read for every sequence's
+context + Q + O + used block-table entries + context lengths) per step time,
+with decode tokens/s/layer beside it.  Device-timed with CUDA events on the
+launching stream; the per-step KV working set is larger than L2, so no flush
+is needed (``--flush-l2`` flushes anyway).  ``e2e`` repeats the step through
+the same C ABI with the per-step inputs copied from pinned host memory and
+the output copied back inside the timed region.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload (the path has no exchange step), value = all ranks' bytes / the
+slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (the reference arm); only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: achieved HBM GB/s (% of B200 peak); decode tokens/s/layer"
+DEFAULT_WORKLOAD = "llama13b"
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_437_b200", "csrc", f)
+                  for f in ("decode.cuh", "ptx.cuh", "pkv_cuda.cu")]
+
+
+# ------------------------------------------------------------------ bytes
+
+def algorithmic_bytes(w) -> dict:
+    """Bytes the step must move at minimum, per the roofline definition:
+    every sequence reads K and V of its whole context for every KV head, plus
+    Q, O, the used block-table entries and the context lengths."""
+    sp = w.spec
+    e = 2  # fp16 / bf16
+    ctx = w.context_lens.astype(np.int64)
+    kv = int(ctx.sum()) * 2 * sp.num_kv_heads * sp.head_dim * e
+    qo = 2 * sp.num_seqs * sp.num_q_heads * sp.head_dim * e
+    used_blocks = -(-ctx // sp.block_size)
+    tables = int(used_blocks.sum()) * 4
+    lens = sp.num_seqs * 4
+    total = kv + qo + tables + lens
+    # shared prefix blocks counted once (their positions are read by every sharer)
+    shared_tokens = 0
+    seen = set()
+    for s in range(sp.num_seqs):
+        for i in range(w.shared_blocks[s]):
+            b = int(w.block_tables[s, i])
+            if b in seen:
+                shared_tokens += sp.block_size
+            seen.add(b)
+    unique_kv = kv - shared_tokens * 2 * sp.num_kv_heads * sp.head_dim * e
+    append = sp.num_seqs * 2 * sp.num_kv_heads * sp.head_dim * e * 2 + sp.num_seqs * 8
+    return dict(total=total, kv=kv, qo=qo, tables=tables, lens=lens,
+                unique_total=unique_kv + qo + tables + lens, append=append)
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
+    return dict(hbm_gbs=6650.0, source="fallback")
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary of this
+    workload, or None when there is none or the kernel changed since."""
+    path = os.path.join(PROFILE_DIR, f"paged_decode_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    mh = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+    mt = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not mh or not mt or mh.group(1) != kernel_hash():
+        return None
+    return int(mt.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def __enter__(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.25)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.tmp is None:
+            return None
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(parts)
+                except ValueError:
+                    continue
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, group=None) -> float:
+    """Max over ranks of a per-rank number (timing only; no data-path exchange)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized():
+        return value
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def weak_scaling_value(bytes_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return bytes_per_rank_step * world * steps / (max_ms * 1e-3) / 1e9
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, rank, world, local):
+    import torch
+
+    import paged_kv_cache_437_b200 as pkv
+    import workloads
+
+    torch.cuda.set_device(local)
+    w = make_workload(args)
+    sp = w.spec
+    dt = torch.float16 if sp.dtype == workloads.F16 else torch.bfloat16
+    nb_bytes = algorithmic_bytes(w)
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).cuda()
+
+    # slots of the new tokens from the library's own host allocator: the pool's
+    # blocks are handed out in the workload's (seeded, shuffled) order by
+    # returning them to the LIFO free list in reverse, then every sequence is
+    # built up to ctx - 1 tokens (prefix blocks shared through fork).
+    alloc = pkv.BlockAllocator(w.num_blocks, sp.block_size)
+    slots_np, alloc_us = allocator_slots(pkv, alloc, w)
+
+    q = dev(w.q)
+    kc, vc = dev(w.k_cache), dev(w.v_cache)
+    kn, vn = dev(w.k_new), dev(w.v_new)
+    slots = torch.from_numpy(slots_np).cuda()
+    tables = torch.from_numpy(np.ascontiguousarray(w.block_tables)).cuda()
+    lens = torch.from_numpy(np.ascontiguousarray(w.context_lens)).cuda()
+    out = torch.empty_like(q)
+    part = args.partition
+    ws = None
+    if part != pkv.PKV_PARTITION_NONE:
+        n = pkv.pkv_decode_workspace_bytes(sp.num_seqs, sp.num_q_heads, sp.num_kv_heads, sp.head_dim,
+                                           w.max_blocks_per_seq * sp.block_size, part)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    merge_launched = part != pkv.PKV_PARTITION_NONE and not (
+        part > 0 and -(-w.max_blocks_per_seq * sp.block_size // part) <= 1)
+    launches_per_step = 2 + (1 if merge_launched else 0)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if args.flush_l2 else None
+
+    def step():
+        pkv.pkv_append(kn, vn, slots, kc, vc, stream)
+        pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pkv.pkv_get_last_error() != pkv.PKV_OK:
+        raise RuntimeError("device check failed during warm-up")
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    step_ev = [(ev(), ev()) for _ in range(args.steps)]
+    dec_ev = [(ev(), ev()) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            step_ev[i][0].record(stream)
+            pkv.pkv_append(kn, vn, slots, kc, vc, stream)
+            dec_ev[i][0].record(stream)
+            pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
+            dec_ev[i][1].record(stream)
+            step_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
+    max_ms = reduce_max(step_ms)
+    if pkv.pkv_get_last_error() != pkv.PKV_OK:
+        raise RuntimeError("device check failed in the timed region")
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None if args.no_e2e else measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out)
+    peaks = load_peaks()
+    ms_per_step = max_ms / args.steps
+    value = weak_scaling_value(nb_bytes["total"], world, args.steps, max_ms)
+    achieved = nb_bytes["total"] / (dec_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": workloads.DTYPE_NAMES[sp.dtype],
+        "data": "synthetic (seeded N(0,1), shapes of the pages' examples)",
+        "config": {
+            "workload": sp.name,
+            "description": sp.description,
+            "num_seqs": sp.num_seqs,
+            "context_tokens_total": int(w.context_lens.sum()),
+            "max_context": int(w.context_lens.max()),
+            "num_q_heads": sp.num_q_heads,
+            "num_kv_heads": sp.num_kv_heads,
+            "head_dim": sp.head_dim,
+            "block_size": sp.block_size,
+            "pool_blocks": w.num_blocks,
+            "partition": {0: "auto (work-balanced)", -1: "none"}.get(part, f"{part} tokens"),
+            "l2": "flushed between steps" if args.flush_l2 else "per-step KV working set > L2 (no flush)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "tokens_per_s_per_layer": round(sp.num_seqs * world / (ms_per_step * 1e-3), 1),
+        "algorithmic_bytes_per_step": nb_bytes["total"],
+        "unique_bytes_per_step": nb_bytes["unique_total"],
+        "frac_of_8TBs": round(value / world / 8000.0, 4),
+        "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "paged_decode_kernel" + ("+lse_merge_kernel" if merge_launched else ""),
+            "achieved": round(achieved, 2),
+            "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"],
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": profiled_traffic(sp.name),
+            "algorithmic_bytes_per_launch": nb_bytes["total"],
+            "us_per_launch": round(dec_ms * 1e3, 3),
+        },
+        "e2e": None if e2e is None else {
+            "value": round(weak_scaling_value(nb_bytes["total"], world, args.steps, e2e["ms"]), 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": e2e["h2d"],
+            "d2h_bytes_per_step": e2e["d2h"],
+            "ms_per_step": round(e2e["ms"] / args.steps, 5),
+        },
+        "allocator_us_per_step": round(alloc_us, 2),
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        result["cpu_baseline"] = cpu_baseline(w, nb_bytes, args.cpu_seconds)
+    alloc.close()
+    return result
+
+
+def _build_sequences(alloc, w):
+    """Create the workload's sequences through the allocator: one holder
+    sequence per sharing group owns the group's prefix blocks, members fork
+    it (refcounted sharing of whole blocks) and grow to ctx - 1 tokens."""
+    sp = w.spec
+    holders = {}
+    if sp.share_group:
+        for s in range(sp.num_seqs):
+            g = s // sp.share_group
+            holders[g] = max(holders.get(g, 0), w.shared_blocks[s])
+        for g in sorted(holders):
+            h = alloc.seq_create()
+            for _ in range(holders[g] * sp.block_size):
+                alloc.append_slot(h)
+            holders[g] = h
+    seqs = []
+    for s in range(sp.num_seqs):
+        if sp.share_group:
+            seq = alloc.seq_fork(holders[s // sp.share_group], w.shared_blocks[s])
+        else:
+            seq = alloc.seq_create()
+        while alloc.context_len(seq) < int(w.context_lens[s]) - 1:
+            alloc.append_slot(seq)
+        seqs.append(seq)
+    return seqs, holders
+
+
+def measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out):
+    """The same step through the C ABI with the per-step inputs in pinned host
+    memory: H2D copies of q, the new K/V, slots, tables and lengths, the
+    kernels, and the D2H copy of the output, all inside the timed region."""
+    import torch
+
+    pin = lambda t: t.cpu().pin_memory()
+    h_q, h_kn, h_vn = pin(q), pin(kn), pin(vn)
+    h_slots, h_tables, h_lens = pin(slots), pin(tables), pin(lens)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_slots, h_tables, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        kn.copy_(h_kn, non_blocking=True)
+        vn.copy_(h_vn, non_blocking=True)
+        slots.copy_(h_slots, non_blocking=True)
+        tables.copy_(h_tables, non_blocking=True)
+        lens.copy_(h_lens, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1))
+    barrier()
+    return dict(ms=e2e_ms, h2d=h2d, d2h=d2h)
+
+
+def allocator_slots(pkv, alloc, w):
+    """Build the workload's tables through the library's host allocator and
+    return the slots of this step's new tokens and the allocator's host time
+    per step (us).  A dry run on a scratch allocator (whose pops come out
+    0, 1, 2, ...) shows which table entry each pop serves; returning the pool
+    to the real allocator's LIFO free list in the reverse of the wanted order
+    then makes its pops reproduce the workload's seeded block assignment."""
+    sp = w.spec
+    scratch = pkv.BlockAllocator(w.num_blocks, sp.block_size)
+    seqs, holders = _build_sequences(scratch, w)
+    scratch.append_slots(seqs)
+    want = {}
+    for s, seq in enumerate(seqs):
+        for i, k in enumerate(scratch.block_table(seq)):
+            want[int(k)] = int(w.block_tables[s, i])
+    scratch.close()
+    order = [want[k] for k in range(len(want))]
+    rest = sorted(set(range(w.num_blocks)) - set(order))
+    got = [alloc.alloc() for _ in range(w.num_blocks)]
+    assert got == list(range(w.num_blocks))
+    for b in reversed(order + rest):
+        alloc.decref(b)
+    seqs, holders = _build_sequences(alloc, w)
+    for h in holders.values():
+        alloc.seq_free(h)
+    t0 = time.perf_counter()
+    slots = alloc.append_slots(seqs)
+    tables, lens = alloc.batch_tables(seqs, w.max_blocks_per_seq)
+    alloc_us = (time.perf_counter() - t0) * 1e6
+    if not (np.array_equal(tables, w.block_tables) and np.array_equal(lens, w.context_lens)):
+        raise RuntimeError("allocator tables differ from the workload's")
+    return slots, alloc_us
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+
+def pair_share_bytes(w, s: int) -> float:
+    """Algorithmic bytes attributable to one (sequence, query head) pair."""
+    sp = w.spec
+    g = sp.num_q_heads // sp.num_kv_heads
+    ctx = int(w.context_lens[s])
+    kv = ctx * 2 * sp.head_dim * 2 / g
+    return kv + 2 * sp.head_dim * 2 + (-(-ctx // sp.block_size) * 4 + 4) / sp.num_q_heads
+
+
+def cpu_baseline(w, nb_bytes, seconds: float) -> dict:
+    import oracle
+
+    sp = w.spec
+    rng = np.random.default_rng(123)
+    pairs_all = np.array([(s, h) for s in range(sp.num_seqs) for h in range(sp.num_q_heads)], dtype=np.int64)
+    rng.shuffle(pairs_all)
+    oracle.load()
+    cores = oracle.num_threads()
+    # pilot to size the sample
+    pilot = pairs_all[:max(1, cores)]
+    t0 = time.perf_counter()
+    oracle.attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, sp.dtype, pairs=pilot)
+    t_pilot = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(len(pairs_all), max(len(pilot), len(pilot) * seconds / t_pilot)))
+    sample = pairs_all[:n]
+    t0 = time.perf_counter()
+    oracle.attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, sp.dtype, pairs=sample)
+    dt = time.perf_counter() - t0
+    done = sum(pair_share_bytes(w, int(s)) for s, _ in sample)
+    return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {len(pairs_all)} (sequence, query head) pairs of {sp.name}, fp64 C oracle "
+                      f"(gather through block tables + two-pass softmax), {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
+def make_workload(args):
+    import dataclasses
+
+    import workloads
+
+    spec = workloads.CONFIGS[args.workload]
+    if args.seqs:
+        n = min(args.seqs, spec.num_seqs)
+        kw = dict(num_seqs=n, name=f"{spec.name}_first{n}")
+        if spec.context_lens is not None:
+            kw["context_lens"] = spec.context_lens[:n]
+        if spec.num_blocks is not None:
+            kw["num_blocks"] = None
+        spec = dataclasses.replace(spec, **kw)
+    return workloads.make(spec)
+
+
+def run_reference(args, rank, world):
+    import oracle
+
+    w = make_workload(args)
+    sp = w.spec
+    nb_bytes = algorithmic_bytes(w)
+    oracle.load()
+    cores = oracle.num_threads()
+    rng = np.random.default_rng(7)
+    pairs_all = np.array([(s, h) for s in range(sp.num_seqs) for h in range(sp.num_q_heads)], dtype=np.int64)
+    rng.shuffle(pairs_all)
+    # each step: a bounded sample, sized so the whole run stays within minutes
+    budget = max(2.0, args.cpu_seconds) / max(1, args.steps + args.warmup)
+    pilot = pairs_all[:max(1, cores)]
+    t0 = time.perf_counter()
+    oracle.attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, sp.dtype, pairs=pilot)
+    t_pilot = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(len(pairs_all), max(len(pilot), len(pilot) * budget / t_pilot)))
+    sample = pairs_all[:n]
+    share = sum(pair_share_bytes(w, int(s)) for s, _ in sample)
+    for _ in range(args.warmup):
+        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, sp.dtype,
+                         pairs=sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, sp.dtype,
+                         pairs=sample)
+    dt = time.perf_counter() - t0
+    value = share * args.steps / dt / 1e9
+    # time per full step, extrapolated from the sample's share of the bytes
+    ms_full = dt / args.steps * (nb_bytes["total"] / share) * 1e3
+    sample_desc = (f"{n} of {len(pairs_all)} (sequence, query head) pairs of {sp.name} per step, fp64 C oracle "
+                   f"on {cores} host threads")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_full, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), shapes of the pages' examples)",
+        "config": {"workload": sp.name, "description": sp.description, "parallelism": "host CPU"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample_desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# ------------------------------------------------------------------ main
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--partition", type=int, default=None,
+                    help="partition tokens: 0 auto (default), -1 none, P > 0 fixed P-token partitions")
+    ap.add_argument("--flush-l2", action="store_true")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass (profiling runs)")
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="run the workload with its first N sequences only (small profiling cases)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.partition is None:
+        import workloads
+
+        args.partition = workloads.CONFIGS[args.workload].partition_tokens or 0
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        result = run_gpu(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -87,7 +87,13 @@ def test_scaling_v_by_two_doubles_output_exactly(mode):
     w2 = workloads.Workload(w.spec, w.context_lens, w.block_tables, w.num_blocks, w.owned_blocks,
                             w.shared_blocks, w.q, kc, vc2, w.k_new, dbl(w.v_new), w.scale)
     out2 = _run(w2, kc, vc2, slots, mode)
-    assert torch.equal(out2, base * 2)
+    # exact wherever the output is a normal fp16 number; in the subnormal range
+    # (|x| < 2^-14) rounding 2x and doubling round(x) can differ by one quantum
+    b2 = (base.double() * 2).cpu()
+    o2 = out2.double().cpu()
+    normal = b2.abs() >= 2.0 ** -13
+    assert torch.equal(o2[normal], b2[normal])
+    assert float((o2 - b2).abs().max()) <= 2.0 ** -24
 
 
 @pytest.mark.parametrize("mode", MODES + [512])
