@@ -58,7 +58,8 @@ typedef enum pkv_status {
     PKV_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed               */
     PKV_ERR_SHARED_WRITE = -4, /* allocator: the target block is shared (refcount>1) */
     PKV_ERR_DEVICE_CHECK = -5, /* a kernel found an index out of range and skipped it */
-    PKV_ERR_TIMEOUT = -6       /* a kernel's bounded wait ran out and it returned early */
+    PKV_ERR_TIMEOUT = -6,      /* a kernel's bounded wait ran out and it returned early */
+    PKV_ERR_SCRATCH_TOO_SMALL = -7 /* the shape needs more scratch than the fixed static area */
 } pkv_status;
 
 typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
@@ -142,6 +143,45 @@ pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_h
                                 const int32_t *context_lens, float scale, void *out,
                                 void *workspace, size_t workspace_bytes,
                                 int32_t partition_tokens, pkv_stream stream);
+
+/* --------------------------------------------------------------------------
+ * pkv_decode_attention_static_scratch -- pkv_decode_attention for callers
+ * that cannot allocate device memory.  (No counterpart on the pages: this is
+ * an interface convenience, not part of the method.)
+ *
+ * Who needs it: code that only ever receives device pointers from its host
+ * framework -- a custom-operator or plugin interface that hands over the
+ * inputs and outputs but no allocator -- and serving loops that forbid device
+ * allocation once they are running, because cudaMalloc / cudaFree can
+ * synchronise the device, fail under memory pressure or fragment the pool in
+ * the middle of a run.  Such callers still pass q, the caches, the tables,
+ * the lengths and out; the split-context scratch comes from a fixed array
+ * that lives in the library's device image.
+ *
+ * Arguments and results are those of pkv_decode_attention with the scratch
+ * taken from a file-scope device array of PKV_STATIC_SCRATCH_BYTES bytes
+ * (every GPU that loads the library holds that array until the process
+ * exits).  A shape whose split scratch (pkv_decode_workspace_bytes for the
+ * same arguments) exceeds it is refused with PKV_ERR_SCRATCH_TOO_SMALL
+ * before anything is launched; PKV_PARTITION_NONE needs no scratch.
+ *
+ * The first call on each device looks up the array's device address (a
+ * runtime query, no allocation) with that device current; make that first
+ * call before any stream capture.  Every call on a device shares the one
+ * array and leaves its last contents there; nothing in it has to start at
+ * zero (each call writes every value it later reads).  Calls whose kernels
+ * overlap on the GPU -- e.g. on two streams at once -- race on the array and
+ * must be serialised by the caller.  No cudaMalloc, cudaFree or allocating
+ * library routine is called.
+ * ------------------------------------------------------------------------ */
+#define PKV_STATIC_SCRATCH_BYTES (32u << 20)
+
+pkv_status pkv_decode_attention_static_scratch(const void *q, int64_t num_seqs, int64_t num_q_heads,
+                                               pkv_cache k_cache, pkv_cache v_cache,
+                                               const int32_t *block_tables,
+                                               int64_t max_blocks_per_seq,
+                                               const int32_t *context_lens, float scale, void *out,
+                                               int32_t partition_tokens, pkv_stream stream);
 
 /* Bytes of workspace pkv_decode_attention needs for this shape and
  * partition_tokens on the CURRENT device (AUTO depends on its SM count).

@@ -23,6 +23,8 @@ PKV_ERR_CUDA = -3
 PKV_ERR_SHARED_WRITE = -4
 PKV_ERR_DEVICE_CHECK = -5
 PKV_ERR_TIMEOUT = -6
+PKV_ERR_SCRATCH_TOO_SMALL = -7
+PKV_STATIC_SCRATCH_BYTES = 32 << 20
 
 PKV_F16 = 0
 PKV_BF16 = 1
@@ -72,6 +74,9 @@ def _load():
         "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "pkv_get_last_error": (ctypes.c_int, []),
         "pkv_test_inject_wait_timeout": (ctypes.c_int, [_c_i32, _c_i64]),
+        "pkv_decode_attention_static_scratch": (ctypes.c_int, [_c_vp, _c_i64, _c_i64, pkv_cache, pkv_cache,
+                                                               _c_vp, _c_i64, _c_vp, ctypes.c_float, _c_vp,
+                                                               _c_i32, _c_vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -180,6 +185,20 @@ def pkv_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale:
 def pkv_test_inject_wait_timeout(enable: bool, wait_limit_ns: int = 50_000_000) -> None:
     _check(lib.pkv_test_inject_wait_timeout(1 if enable else 0, int(wait_limit_ns)),
            "pkv_test_inject_wait_timeout")
+
+
+def pkv_decode_attention_static_scratch(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                                        partition_tokens: int = PKV_PARTITION_AUTO, stream=None) -> None:
+    """pkv_decode_attention for callers that cannot allocate device memory:
+    the split scratch is the library's fixed device array (see include/pkv.h).
+    Calls that overlap on the GPU share that array and must be serialised."""
+    for t, n in ((q, "q"), (out, "out"), (block_tables, "block_tables"), (context_lens, "context_lens")):
+        _require(t, n)
+    st = lib.pkv_decode_attention_static_scratch(q.data_ptr(), q.shape[0], q.shape[1], cache_desc(k_cache),
+                                                 cache_desc(v_cache), block_tables.data_ptr(),
+                                                 block_tables.shape[1], context_lens.data_ptr(), float(scale),
+                                                 out.data_ptr(), int(partition_tokens), _stream_ptr(stream))
+    _check(st, "pkv_decode_attention_static_scratch")
 
 
 def pkv_get_last_error() -> int:

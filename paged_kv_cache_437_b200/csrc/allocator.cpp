@@ -275,6 +275,7 @@ const char *pkv_status_string(pkv_status s) {
     case PKV_ERR_SHARED_WRITE: return "write into a shared block";
     case PKV_ERR_DEVICE_CHECK: return "device-side index check failed";
     case PKV_ERR_TIMEOUT: return "device wait timed out";
+    case PKV_ERR_SCRATCH_TOO_SMALL: return "shape needs more than the static scratch";
     }
     return "unknown status";
 }

@@ -439,4 +439,69 @@ pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns) {
     return PKV_OK;
 }
 
+
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without any device allocation by the caller or by us.
+//
+// Some callers cannot allocate device memory: a plugin or custom-operator
+// interface that only receives device pointers for its inputs and outputs,
+// or a serving loop that bans cudaMalloc after start-up (it can synchronise
+// the device, fail under pressure or fragment memory mid-run).  For them the
+// split-context scratch lives in this fixed file-scope array instead of a
+// caller-provided workspace.  Every GPU that loads the library keeps it for
+// the life of the process, so its size is kept modest.
+static __device__ __align__(256) unsigned char g_static_scratch[PKV_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// In host code `g_static_scratch` names a host-side shadow, not device
+// memory: the device address has to be asked for, once per device, with that
+// device current.  Returns nullptr if the runtime cannot provide it.
+void *static_scratch_device_ptr() {
+    static void *addr[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess)
+            return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" pkv_status pkv_decode_attention_static_scratch(
+    const void *q, int64_t num_seqs, int64_t num_q_heads, pkv_cache k_cache, pkv_cache v_cache,
+    const int32_t *block_tables, int64_t max_blocks_per_seq, const int32_t *context_lens, float scale,
+    void *out, int32_t partition_tokens, pkv_stream stream) {
+    if (partition_tokens == PKV_PARTITION_NONE)
+        return pkv_decode_attention(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables,
+                                    max_blocks_per_seq, context_lens, scale, out, nullptr, 0,
+                                    partition_tokens, stream);
+    if (num_seqs == 0)
+        return pkv_decode_attention(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables,
+                                    max_blocks_per_seq, context_lens, scale, out, nullptr, 0,
+                                    partition_tokens, stream);
+    if (!cache_ok(k_cache) || max_blocks_per_seq <= 0)
+        return PKV_ERR_INVALID;
+    const size_t need = pkv_decode_workspace_bytes(
+        num_seqs, num_q_heads, k_cache.num_kv_heads, k_cache.head_dim,
+        max_blocks_per_seq * k_cache.block_size, partition_tokens);
+    if (need == 0)
+        return PKV_ERR_INVALID;  // shape rejected (or no device to size it on)
+    if (need > (size_t)PKV_STATIC_SCRATCH_BYTES)
+        return PKV_ERR_SCRATCH_TOO_SMALL;
+    void *scratch = static_scratch_device_ptr();
+    if (!scratch)
+        return PKV_ERR_CUDA;
+    return pkv_decode_attention(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables,
+                                max_blocks_per_seq, context_lens, scale, out, scratch,
+                                (size_t)PKV_STATIC_SCRATCH_BYTES, partition_tokens, stream);
+}
