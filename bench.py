@@ -3,9 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--partition P] [--flush-l2] [--impl reference]
 
-A step is the whole hot path on one batch: pkv_append of every sequence's new
-token, then pkv_decode_attention (decode kernel + log-sum-exp merge when the
-schedule splits contexts).  Inputs are synthetic and seeded (``workloads``),
+A step is the whole hot path on one batch: the append of every sequence's new
+token and the attention (decode kernel + log-sum-exp merge when the schedule
+splits contexts), by default through the fused pkv_append_decode_attention
+call (``--unfused``: pkv_append then pkv_decode_attention).  Inputs are synthetic and seeded (``workloads``),
 shaped like the pages' examples; the default workload is the 13B-shaped layer
 (32 sequences x 2048 context, 40/40 heads, D 128, block 16, fp16).
 
@@ -243,14 +244,37 @@ def run_gpu(args, rank, world, local):
         ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
     merge_launched = part != pkv.PKV_PARTITION_NONE and not (
         part > 0 and -(-w.max_blocks_per_seq * sp.block_size // part) <= 1)
-    launches_per_step = 2 + (1 if merge_launched else 0)
+    launches_per_step = (1 if not args.unfused else 2) + (1 if merge_launched else 0)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if args.flush_l2 else None
 
-    def step():
-        pkv.pkv_append(kn, vn, slots, kc, vc, stream)
-        pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
+    # the C ABI calls with their arguments marshalled once (the Python
+    # binding's checks ran above; the timed loops make the raw calls)
+    import ctypes
 
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    kdesc, vdesc = pkv.cache_desc(kc), pkv.cache_desc(vc)
+    append_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr(), slots.numel(), kdesc, vdesc, sptr)
+    ws_ptr = ws.data_ptr() if ws is not None else None
+    ws_bytes = ws.numel() if ws is not None else 0
+    decode_args = (q.data_ptr(), q.shape[0], q.shape[1], kdesc, vdesc, tables.data_ptr(), tables.shape[1],
+                   lens.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, part, sptr)
+    c_append, c_decode = pkv.lib.pkv_append, pkv.lib.pkv_decode_attention
+    c_fused = pkv.lib.pkv_append_decode_attention
+    fused_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr()) + decode_args
+
+    if args.unfused:
+        def step():
+            c_append(*append_args)
+            c_decode(*decode_args)
+    else:
+        def step():
+            c_fused(*fused_args)
+
+    # the binding path once, with its argument checks
+    pkv.pkv_append(kn, vn, slots, kc, vc, stream)
+    pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
+    pkv.pkv_append_decode_attention(kn, vn, slots, q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -258,24 +282,44 @@ def run_gpu(args, rank, world, local):
         raise RuntimeError("device check failed during warm-up")
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    step_ev = [(ev(), ev()) for _ in range(args.steps)]
-    dec_ev = [(ev(), ev()) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        # K whole steps, events only around the region (no events between the
+        # kernels, so each launch can overlap the previous kernel's tail)
+        t0, t1 = ev(), ev()
+        t0.record(stream)
         for i in range(args.steps):
             if flush is not None:
                 flush.zero_()
-            step_ev[i][0].record(stream)
-            pkv.pkv_append(kn, vn, slots, kc, vc, stream)
-            dec_ev[i][0].record(stream)
-            pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
-            dec_ev[i][1].record(stream)
-            step_ev[i][1].record(stream)
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        step_ms = t0.elapsed_time(t1)
+        # the dominant kernel: K launches of the decode kernel (the fused
+        # append + decode call of the step, or the decode call alone) back to
+        # back, plus its merge when contexts are split
+        d0, d1 = ev(), ev()
+        d0.record(stream)
+        for i in range(args.steps):
+            if args.unfused:
+                c_decode(*decode_args)
+            else:
+                c_fused(*fused_args)
+        d1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    step_ms = sum(a.elapsed_time(b) for a, b in step_ev)
-    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
+    dec_ms = d0.elapsed_time(d1) / args.steps
+    if flush is not None:
+        # the flush runs inside the step region: subtract its own time
+        f0, f1 = ev(), ev()
+        f0.record(stream)
+        for _ in range(args.steps):
+            flush.zero_()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        step_ms -= f0.elapsed_time(f1)
     max_ms = reduce_max(step_ms)
     if pkv.pkv_get_last_error() != pkv.PKV_OK:
         raise RuntimeError("device check failed in the timed region")
@@ -313,6 +357,7 @@ def run_gpu(args, rank, world, local):
             "partition": {0: "auto (work-balanced)", -1: "none"}.get(part, f"{part} tokens"),
             "l2": "flushed between steps" if args.flush_l2 else "per-step KV working set > L2 (no flush)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "step_call": "pkv_append + pkv_decode_attention" if args.unfused else "pkv_append_decode_attention",
         },
         "tokens_per_s_per_layer": round(sp.num_seqs * world / (ms_per_step * 1e-3), 1),
         "algorithmic_bytes_per_step": nb_bytes["total"],
@@ -571,6 +616,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass (profiling runs)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="step = pkv_append + pkv_decode_attention (default: pkv_append_decode_attention)")
     ap.add_argument("--seqs", type=int, default=None,
                     help="run the workload with its first N sequences only (small profiling cases)")
     args = ap.parse_args(argv)

@@ -145,6 +145,33 @@ pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_h
                                 int32_t partition_tokens, pkv_stream stream);
 
 /* --------------------------------------------------------------------------
+ * pkv_append_decode_attention -- pkv_append and pkv_decode_attention of one
+ * decode step in a single kernel launch (plus the merge launch when contexts
+ * are split).  Same arguments as pkv_decode_attention, plus:
+ *
+ *   k_new, v_new   device [B][Hkv][D]: the new token of sequence s is row s
+ *   slot_mapping   device int64 [B]: its slot, which must be the slot of
+ *                  position context_lens[s] - 1 of sequence s (what
+ *                  pkv_seq_append_slot returned); < 0 means no new token
+ *
+ * Result: identical to pkv_append(k_new, v_new, slot_mapping, B, ...)
+ * followed by pkv_decode_attention(...) under that precondition.  The warp
+ * that owns a sequence's last position reads the new row from k_new / v_new,
+ * stores it in the cache and uses it directly, so no separate launch (and no
+ * ordering between the two) is needed.  A sequence with context_lens[s] == 0
+ * has no attended position and its token is not written.  For any other
+ * token layout (several tokens per sequence, slots not at the last
+ * position) use the two separate calls.
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_append_decode_attention(const void *k_new, const void *v_new,
+                                       const int64_t *slot_mapping, const void *q, int64_t num_seqs,
+                                       int64_t num_q_heads, pkv_cache k_cache, pkv_cache v_cache,
+                                       const int32_t *block_tables, int64_t max_blocks_per_seq,
+                                       const int32_t *context_lens, float scale, void *out,
+                                       void *workspace, size_t workspace_bytes,
+                                       int32_t partition_tokens, pkv_stream stream);
+
+/* --------------------------------------------------------------------------
  * pkv_decode_attention_static_scratch -- pkv_decode_attention for callers
  * that cannot allocate device memory.  (No counterpart on the pages: this is
  * an interface convenience, not part of the method.)
@@ -253,6 +280,10 @@ pkv_status pkv_batch_tables(void *h, const int32_t *seqs, int32_t n, int32_t *ds
  * enable == 0 restores normal operation (2 s limit).  Host-side setting only;
  * nothing faults, traps or hangs. */
 pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns);
+
+/* Text of the last CUDA runtime error a call of this thread reported as
+ * PKV_ERR_CUDA ("no error" if none); static storage. */
+const char *pkv_last_cuda_error(void);
 
 /* Human-readable name of a status code (static storage). */
 const char *pkv_status_string(pkv_status s);

@@ -43,7 +43,8 @@ class pkv_cache(ctypes.Structure):
 
 class PkvError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {pkv_status_string(status)} ({status})")
+        detail = f" [{lib.pkv_last_cuda_error().decode()}]" if status == PKV_ERR_CUDA else ""
+        super().__init__(f"{what}: {pkv_status_string(status)} ({status}){detail}")
         self.status = status
 
 
@@ -56,6 +57,9 @@ def _load():
         "pkv_decode_attention": (ctypes.c_int, [_c_vp, _c_i64, _c_i64, pkv_cache, pkv_cache, _c_vp, _c_i64,
                                                 _c_vp, ctypes.c_float, _c_vp, _c_vp, _c_sz, _c_i32, _c_vp]),
         "pkv_decode_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i32]),
+        "pkv_append_decode_attention": (ctypes.c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, pkv_cache,
+                                                       pkv_cache, _c_vp, _c_i64, _c_vp, ctypes.c_float, _c_vp,
+                                                       _c_vp, _c_sz, _c_i32, _c_vp]),
         "pkv_alloc_create": (ctypes.c_int, [_c_i32, _c_i32, ctypes.POINTER(_c_vp)]),
         "pkv_alloc_destroy": (None, [_c_vp]),
         "pkv_block_alloc": (ctypes.c_int, [_c_vp, ctypes.POINTER(_c_i32)]),
@@ -72,6 +76,7 @@ def _load():
         "pkv_seq_context_len": (_c_i64, [_c_vp, _c_i32]),
         "pkv_batch_tables": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_i32, _c_vp]),
         "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "pkv_last_cuda_error": (ctypes.c_char_p, []),
         "pkv_get_last_error": (ctypes.c_int, []),
         "pkv_test_inject_wait_timeout": (ctypes.c_int, [_c_i32, _c_i64]),
         "pkv_decode_attention_static_scratch": (ctypes.c_int, [_c_vp, _c_i64, _c_i64, pkv_cache, pkv_cache,
@@ -199,6 +204,36 @@ def pkv_decode_attention_static_scratch(q, k_cache, v_cache, block_tables, conte
                                                  block_tables.shape[1], context_lens.data_ptr(), float(scale),
                                                  out.data_ptr(), int(partition_tokens), _stream_ptr(stream))
     _check(st, "pkv_decode_attention_static_scratch")
+
+
+def pkv_append_decode_attention(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens,
+                                scale: float, out, workspace=None, partition_tokens: int = PKV_PARTITION_AUTO,
+                                stream=None) -> None:
+    """Append (one new token per sequence, at position ctx-1) and decode in one launch."""
+    import torch
+
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (slot_mapping, "slot_mapping"), (q, "q"), (out, "out"),
+                 (block_tables, "block_tables"), (context_lens, "context_lens")):
+        _require(t, n)
+    if slot_mapping.dtype != torch.int64 or block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("slot_mapping int64, block_tables / context_lens int32")
+    if q.dtype != k_cache.dtype or out.dtype != q.dtype or k_new.dtype != q.dtype or v_new.dtype != q.dtype:
+        raise TypeError("q, out, k_new, v_new and the caches must share one dtype")
+    b = q.shape[0]
+    if k_new.shape != (b, k_cache.shape[1], k_cache.shape[3]) or v_new.shape != k_new.shape or \
+            slot_mapping.numel() != b or out.shape != q.shape or block_tables.shape[0] != b or \
+            context_lens.numel() != b:
+        raise ValueError("shapes: k_new/v_new [B][Hkv][D], slot_mapping [B], q/out [B][Hq][D]")
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        _require(workspace, "workspace")
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = lib.pkv_append_decode_attention(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(), q.data_ptr(),
+                                         b, q.shape[1], cache_desc(k_cache), cache_desc(v_cache),
+                                         block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+                                         float(scale), out.data_ptr(), ws_ptr or None, ws_bytes,
+                                         int(partition_tokens), _stream_ptr(stream))
+    _check(st, "pkv_append_decode_attention")
 
 
 def pkv_get_last_error() -> int:

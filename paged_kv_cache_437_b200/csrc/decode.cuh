@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <climits>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -43,7 +44,7 @@ namespace pkv {
 constexpr int kTileTokens = 16;                        // tokens per MMA k-step / TMA box rows
 constexpr int kBoxCols = 64;                           // 16-bit elements per box row (128 B)
 constexpr int kBoxBytes = kBoxCols * 2 * kTileTokens;  // 2048
-constexpr int kMaxRows = 16;                           // query heads per unit (MMA M)
+constexpr int kMaxRows = 16;                           // max query heads per unit (MMA N, 1 or 2 n-tiles)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;       // 2 s bound on every wait
 
 // device error word bits
@@ -61,7 +62,7 @@ struct DecodeArgs {
     const int32_t *context_lens;   // [B]
     int64_t mb;                    // MB
     int64_t nb;                    // NB
-    int B, Hq, Hkv, G, n_hg, npairs, bs;
+    int B, Hq, Hkv, G, n_hg, npairs, bs;  // n_hg = ceil(G / heads per unit)
     float scale_log2;              // scale * log2(e)
     int mode;
     int part_tiles;                // partition mode: tiles per partition
@@ -75,6 +76,13 @@ struct DecodeArgs {
     unsigned *err;
     uint64_t wait_limit_ns;        // bound on every mbarrier wait
     int inject_no_issue;           // testing: issue no copies so that waits run out
+    // fused append (pkv_append_decode_attention), all null otherwise: token s
+    // is sequence s's new token, at position context_lens[s] - 1, slot slots[s]
+    const uint16_t *k_new;         // [B][Hkv][D]
+    const uint16_t *v_new;
+    const int64_t *slots;          // [B], < 0: no append for that sequence
+    uint16_t *k_cache, *v_cache;   // the pools, for the generic-store append
+    int64_t pool_slots;            // NB * bs
 };
 
 struct SmemLayout {
@@ -231,14 +239,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 
 // ------------------------------------------------------------- decode kernel
 
-template <int D, bool BF16, bool TWO>
+template <int D, bool BF16, int NT>
 __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     constexpr int kTile = kTileTokens * D * 2;  // bytes of one K (or V) tile
-    constexpr int kKSteps = D / 16;
-    constexpr int kNTiles = D / 8;
+    constexpr int kMT = D / 16;                 // k-steps of Q K^T == 16-row d tiles of P V
+    constexpr int HPU = 8 * NT;                 // query heads per unit (MMA N)
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
@@ -265,6 +273,10 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         fence_mbar_init();
         fence_proxy_async_smem();
     }
+    // everything above overlaps the previous kernel (the append); every read
+    // of an input comes after this point
+    griddep_wait();
+    griddep_launch_dependents();
 
     // ---- schedule prologue: per-sequence unit counts and their prefix sums
     if (need_prefix) {
@@ -320,13 +332,33 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 o[i] = make_uint4(0, 0, 0, 0);
         }
         if (a.mode == kModeBalanced && blockIdx.x == 0) {
-            for (int i = threadIdx.x; i <= a.B; i += blockDim.x)
+            // the merge kernel reads the schedule back, plus an upper bound
+            // on the pieces any (sequence, head group) is split into
+            __shared__ int s_ntmax;
+            if (threadIdx.x == 0)
+                s_ntmax = 0;
+            __syncthreads();
+            int ntmax = 0;
+            for (int i = threadIdx.x; i <= a.B; i += blockDim.x) {
                 a.prefix_out[i] = prefix[i];
+                if (i < a.B)
+                    ntmax = max(ntmax, prefix[i + 1] - prefix[i]);
+            }
+            atomicMax(&s_ntmax, ntmax);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                // nt consecutive tiles touch at most ceil(nt * W / T) + 1 warps
+                // (empty-range warps in between included)
+                const long long T = max((long long)prefix[a.B] * a.npairs, 1LL);
+                const long long W = a.total_warps;
+                const long long bound = ((long long)s_ntmax * W + T - 1) / T + 1;
+                a.prefix_out[a.B + 1] = (int)min(bound, (long long)INT_MAX);
+            }
         }
     }
 
-    const int c4 = lane & 3;   // thread-in-quad
-    const int g8 = lane >> 2;  // quad index (MMA row / column group)
+    const int c4 = lane & 3;   // thread-in-quad (MMA column pair)
+    const int g8 = lane >> 2;  // quad index (MMA row)
 
     // ---- producer state (whole warp runs it; lane 0 issues the copies)
     Walker pw;
@@ -339,7 +371,29 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         p_has = false;
     int p_t = p_has ? ps.t0 : 0;
     int tb_seq = -1, tb_base = 0, tb_val = 0;  // lane i caches table entry tb_base + i
+    int nx_seq = -1, nx_base = 0, nx_val = 0;  // the same, prefetched for the next unit
     int issued = 0;
+
+    // Start loading the first 32 table entries of the unit after the current
+    // one, so that entering it does not stall the warp on a dependent load.
+    auto prefetch_next_chunk = [&]() {
+        Walker tmp = pw;
+        Seg ns;
+        bool has = walker_next(tmp, ns, a, prefix, ctxs, gw);
+        while (has && ns.t0 >= ns.t1)
+            has = walker_next(tmp, ns, a, prefix, ctxs, gw);
+        nx_seq = -1;
+        if (has) {
+            const int lb = ns.t0 * kTileTokens / a.bs;
+            const int nblk = ceil_div_i(ns.ctx, a.bs);
+            nx_seq = ns.seq;
+            nx_base = lb;
+            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.seq * a.mb + lb + lane) : 0;
+        }
+    };
+    // set when the producer enters a unit; the prefetch for the unit after it
+    // is issued once this unit's own first chunk is in hand
+    bool want_prefetch = p_has;
 
     auto issue = [&](int stage) {
         const int pos0 = p_t * kTileTokens;
@@ -348,8 +402,17 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         if (ps.seq != tb_seq || lb < tb_base || lb >= tb_base + 32) {
             tb_seq = ps.seq;
             tb_base = lb;
-            const int nblk = ceil_div_i(ps.ctx, a.bs);
-            tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.seq * a.mb + lb + lane) : 0;
+            if (ps.seq == nx_seq && lb == nx_base) {
+                tb_val = nx_val;
+                nx_seq = -1;
+            } else {
+                const int nblk = ceil_div_i(ps.ctx, a.bs);
+                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.seq * a.mb + lb + lane) : 0;
+            }
+        }
+        if (want_prefetch) {
+            want_prefetch = false;
+            prefetch_next_chunk();
         }
         int blk = __shfl_sync(FULL, tb_val, lb - tb_base);
         if (blk < 0 || (int64_t)blk >= a.nb) {
@@ -375,6 +438,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 p_has = walker_next(pw, ps, a, prefix, ctxs, gw);
             } while (p_has && ps.t0 >= ps.t1);
             p_t = p_has ? ps.t0 : 0;
+            want_prefetch = p_has;
         }
     };
 
@@ -382,6 +446,11 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         issue(s);
 
     // ---- consumer
+    // Per 16-token tile, with the tokens as the M rows of the MMA:
+    //   S^T[16 tok][HPU heads] = K[16 tok][D] * Q^T[D][HPU]         (kMT k-steps)
+    //   O^T[D][HPU]          += V^T[D][16 tok] * P^T[16 tok][HPU]   (kMT m-tiles)
+    // P^T comes out of the first product in accumulator layout; one movmatrix
+    // per 8x8 block turns it into the B operand of the second.
     Walker cw;
     Seg cs;
     walker_init(cw, a, prefix, gw);
@@ -390,33 +459,81 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
     int consumed = 0;
     bool failed = false;
 
-    while (!failed && walker_next(cw, cs, a, prefix, ctxs, gw)) {
-        const int kvh = cs.pair / a.n_hg;
-        const int hg = cs.pair - kvh * a.n_hg;
-        const int h0 = kvh * a.G + hg * kMaxRows;
-        const int rows = min(kMaxRows, a.G - hg * kMaxRows);
-
-        // Q fragments (A operand, rows = query heads, k = head dim)
-        uint32_t qa[kKSteps][4];
-        {
-            const uint32_t *qlo = reinterpret_cast<const uint32_t *>(a.q + ((size_t)cs.seq * a.Hq + h0 + g8) * D);
-            const uint32_t *qhi = reinterpret_cast<const uint32_t *>(a.q + ((size_t)cs.seq * a.Hq + h0 + g8 + 8) * D);
-            const bool vlo = g8 < rows;
-            const bool vhi = TWO && (g8 + 8 < rows);
+    // Per-unit inputs -- the query fragments and, for a fused append, the new
+    // token's row and slot -- are loaded one unit ahead: the loads for unit
+    // u+1 are issued when unit u starts and first used when u+1 starts.
+    struct UnitIn {
+        uint32_t qb[NT][kMT][2];  // Q^T as the B operand (k = head dim, n = query head)
+        bool has_new;             // this unit holds its sequence's last position
+        int64_t slot;
+        uint2 kn, vn;
+    };
+    auto load_unit = [&](const Seg &u, UnitIn &in) {
+        const int kvh_u = u.pair / a.n_hg;
+        const int hg_u = u.pair - kvh_u * a.n_hg;
+        const int h0_u = kvh_u * a.G + hg_u * HPU;
+        const int rows_u = min(HPU, a.G - hg_u * HPU);
 #pragma unroll
-            for (int ks = 0; ks < kKSteps; ++ks) {
-                qa[ks][0] = vlo ? __ldg(qlo + ks * 8 + c4) : 0u;
-                qa[ks][2] = vlo ? __ldg(qlo + ks * 8 + 4 + c4) : 0u;
-                qa[ks][1] = vhi ? __ldg(qhi + ks * 8 + c4) : 0u;
-                qa[ks][3] = vhi ? __ldg(qhi + ks * 8 + 4 + c4) : 0u;
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = nt * 8 + g8;
+            const bool valid = head < rows_u;
+            const uint32_t *qr = reinterpret_cast<const uint32_t *>(
+                a.q + ((size_t)u.seq * a.Hq + h0_u + (valid ? head : 0)) * D);
+#pragma unroll
+            for (int ks = 0; ks < kMT; ++ks) {
+                in.qb[nt][ks][0] = valid ? __ldg(qr + ks * 8 + c4) : 0u;
+                in.qb[nt][ks][1] = valid ? __ldg(qr + ks * 8 + 4 + c4) : 0u;
             }
         }
+        in.has_new = a.k_new != nullptr && u.t1 > u.t0 && u.t1 * kTileTokens >= u.ctx;
+        in.slot = -1;
+        in.kn = in.vn = make_uint2(0, 0);
+        if (in.has_new) {
+            in.slot = __ldg(a.slots + u.seq);
+            if (lane < D / 4) {
+                const size_t src = ((size_t)u.seq * a.Hkv + kvh_u) * D;
+                in.kn = __ldg(reinterpret_cast<const uint2 *>(a.k_new + src) + lane);
+                in.vn = __ldg(reinterpret_cast<const uint2 *>(a.v_new + src) + lane);
+            }
+        }
+    };
 
-        float o[kNTiles][4];
+    bool c_has = walker_next(cw, cs, a, prefix, ctxs, gw);
+    UnitIn cur;
+    if (c_has)
+        load_unit(cs, cur);
+    while (!failed && c_has) {
+        const int kvh = cs.pair / a.n_hg;
+        const int hg = cs.pair - kvh * a.n_hg;
+        const int h0 = kvh * a.G + hg * HPU;
+        const int rows = min(HPU, a.G - hg * HPU);
+
+        // issue the next unit's loads now; they land while this unit runs
+        Walker nw = cw;
+        Seg ns;
+        const bool n_has = walker_next(nw, ns, a, prefix, ctxs, gw);
+        UnitIn nxt;
+        if (n_has)
+            load_unit(ns, nxt);
+
+        // Fused append: the unit that holds the sequence's last position
+        // patches the new K/V row into its shared-memory tile at the last
+        // tile and stores it to its cache slot in the epilogue (once per KV
+        // head: head group 0).
+        const bool has_new = cur.has_new;
+        const int64_t new_slot = cur.slot;
+        const uint2 kn2 = cur.kn, vn2 = cur.vn;
+
+        float o[NT][kMT][4];
+        float m_run[NT][2], l_run[NT][2];
 #pragma unroll
-        for (int j = 0; j < kNTiles; ++j)
-            o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-        float m_lo = -INFINITY, l_lo = 0.f, m_hi = -INFINITY, l_hi = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt)
+                o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+            m_run[nt][0] = m_run[nt][1] = -INFINITY;
+            l_run[nt][0] = l_run[nt][1] = 0.f;
+        }
 
         for (int t = cs.t0; t < cs.t1; ++t) {
             const uint32_t bar = bar_base + stage * 8;
@@ -432,93 +549,101 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const uint32_t kb = ring_base + stage * 2 * kTile;
             const uint32_t vb = kb + kTile;
             const int nvalid = min(kTileTokens, cs.ctx - t * kTileTokens);
+            if (has_new && t == cs.t1 - 1 && new_slot >= 0 && new_slot < a.pool_slots) {
+                // the new token's row of this tile, in the 128-byte swizzle
+                const int r = cs.ctx - 1 - t * kTileTokens;
+                if (lane < D / 4) {
+                    const int chunk = lane >> 1;  // 16-byte chunk of the row
+                    const uint32_t off = (chunk >> 3) * kBoxBytes + r * 128 +
+                                         ((uint32_t)((chunk & 7) ^ (r & 7)) << 4) + (lane & 1) * 8;
+                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(kb + off), "r"(kn2.x), "r"(kn2.y)
+                                 : "memory");
+                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(vb + off), "r"(vn2.x), "r"(vn2.y)
+                                 : "memory");
+                }
+                __syncwarp();
+            }
 
-            // S^T tile: rows = query heads, columns = 16 tokens (two n-tiles of 8)
-            float sc[2][4];
+            // S^T = K Q^T
+            float sc[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
                 sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-            for (int kc = 0; kc < D / 32; ++kc) {
+            for (int ks = 0; ks < kMT; ++ks) {
+                const int mi = lane >> 3;
+                const int tok = (lane & 7) + 8 * (mi & 1);
+                const int chunk = 2 * ks + (mi >> 1);
+                const uint32_t addr = kb + (chunk >> 3) * kBoxBytes + tok * 128 +
+                                      ((uint32_t)((chunk & 7) ^ (tok & 7)) << 4);
+                uint32_t ka[4];
+                ldmatrix_x4(addr, ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int row = nt * 8 + (lane & 7);
-                    const int chunk = kc * 4 + (lane >> 3);
-                    const uint32_t addr = kb + (chunk >> 3) * kBoxBytes + row * 128 +
-                                          ((uint32_t)((chunk & 7) ^ (row & 7)) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(addr, b0, b1, b2, b3);
-                    mma_16816<BF16>(sc[nt], qa[2 * kc], b0, b1);
-                    mma_16816<BF16>(sc[nt], qa[2 * kc + 1], b2, b3);
-                }
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_16816<BF16>(sc[nt], ka, cur.qb[nt][ks][0], cur.qb[nt][ks][1]);
             }
 
-            // online softmax (log2 domain)
+            // online softmax per query head (one column of S^T), log2 domain;
+            // this thread holds tokens g8, g8+8 of heads 2*c4, 2*c4+1
+            const bool v_lo = g8 < nvalid;
+            const bool v_hi = g8 + 8 < nvalid;
+            uint32_t pb[NT][2];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < NT; ++nt) {
+                const float x0 = v_lo ? sc[nt][0] * a.scale_log2 : -INFINITY;
+                const float x1 = v_lo ? sc[nt][1] * a.scale_log2 : -INFINITY;
+                const float x2 = v_hi ? sc[nt][2] * a.scale_log2 : -INFINITY;
+                const float x3 = v_hi ? sc[nt][3] * a.scale_log2 : -INFINITY;
+                float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int tok = nt * 8 + 2 * c4 + (i & 1);
-                    const float v = sc[nt][i] * a.scale_log2;
-                    sc[nt][i] = tok < nvalid ? v : -INFINITY;
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
                 }
-            }
-            float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-            const float mnew = fmaxf(m_lo, mx);
-            const float alpha = exp2f(m_lo - mnew);
-            m_lo = mnew;
-            float p00 = exp2f(sc[0][0] - mnew), p01 = exp2f(sc[0][1] - mnew);
-            float p10 = exp2f(sc[1][0] - mnew), p11 = exp2f(sc[1][1] - mnew);
-            l_lo = l_lo * alpha + ((p00 + p01) + (p10 + p11));
-            float alpha_hi = 1.f, q00 = 0.f, q01 = 0.f, q10 = 0.f, q11 = 0.f;
-            if constexpr (TWO) {
-                float mh = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-                mh = fmaxf(mh, __shfl_xor_sync(FULL, mh, 1));
-                mh = fmaxf(mh, __shfl_xor_sync(FULL, mh, 2));
-                const float mnh = fmaxf(m_hi, mh);
-                alpha_hi = exp2f(m_hi - mnh);
-                m_hi = mnh;
-                q00 = exp2f(sc[0][2] - mnh);
-                q01 = exp2f(sc[0][3] - mnh);
-                q10 = exp2f(sc[1][2] - mnh);
-                q11 = exp2f(sc[1][3] - mnh);
-                l_hi = l_hi * alpha_hi + ((q00 + q01) + (q10 + q11));
-            }
+                const float mn0 = fmaxf(m_run[nt][0], mx0);
+                const float mn1 = fmaxf(m_run[nt][1], mx1);
+                const float al0 = exp2f(m_run[nt][0] - mn0);
+                const float al1 = exp2f(m_run[nt][1] - mn1);
+                m_run[nt][0] = mn0;
+                m_run[nt][1] = mn1;
+                const float p0 = exp2f(x0 - mn0), p2 = exp2f(x2 - mn0);
+                const float p1 = exp2f(x1 - mn1), p3 = exp2f(x3 - mn1);
+                l_run[nt][0] = l_run[nt][0] * al0 + (p0 + p2);
+                l_run[nt][1] = l_run[nt][1] * al1 + (p1 + p3);
 #pragma unroll
-            for (int j = 0; j < kNTiles; ++j) {
-                o[j][0] *= alpha;
-                o[j][1] *= alpha;
-                if constexpr (TWO) {
-                    o[j][2] *= alpha_hi;
-                    o[j][3] *= alpha_hi;
+                for (int mt = 0; mt < kMT; ++mt) {
+                    o[nt][mt][0] *= al0;
+                    o[nt][mt][2] *= al0;
+                    o[nt][mt][1] *= al1;
+                    o[nt][mt][3] *= al1;
                 }
+                pb[nt][0] = movmatrix_trans(pack2<BF16>(p0, p1));  // tokens 0-7
+                pb[nt][1] = movmatrix_trans(pack2<BF16>(p2, p3));  // tokens 8-15
             }
-            uint32_t pa[4];
-            pa[0] = pack2<BF16>(p00, p01);
-            pa[1] = TWO ? pack2<BF16>(q00, q01) : 0u;
-            pa[2] = pack2<BF16>(p10, p11);
-            pa[3] = TWO ? pack2<BF16>(q10, q11) : 0u;
 
-            // positions past the context may hold anything (even NaN): zero
-            // their V so that 0 * V stays 0 in the MMA
+            // O^T += V^T P^T.  Positions past the context may hold anything
+            // (even NaN): zero their V so that 0 * V stays 0 in the MMA.
             uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
             if (nvalid < kTileTokens) {
                 m01 = (2 * c4 < nvalid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < nvalid ? 0xffff0000u : 0u);
                 m23 = (2 * c4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < nvalid ? 0xffff0000u : 0u);
             }
 #pragma unroll
-            for (int jj = 0; jj < D / 16; ++jj) {
+            for (int mt = 0; mt < kMT; ++mt) {
                 const int mi = lane >> 3;
-                const int tok = (lane & 7) + 8 * (mi & 1);
-                const int chunk = 2 * jj + (mi >> 1);
+                const int tok = (lane & 7) + 8 * (mi >> 1);
+                const int chunk = 2 * mt + (mi & 1);
                 const uint32_t addr = vb + (chunk >> 3) * kBoxBytes + tok * 128 +
                                       ((uint32_t)((chunk & 7) ^ (tok & 7)) << 4);
-                uint32_t v0, v1, v2, v3;
-                ldmatrix_x4_trans(addr, v0, v1, v2, v3);
-                mma_16816<BF16>(o[2 * jj], pa, v0 & m01, v1 & m23);
-                mma_16816<BF16>(o[2 * jj + 1], pa, v2 & m01, v3 & m23);
+                uint32_t va[4];
+                ldmatrix_x4_trans(addr, va[0], va[1], va[2], va[3]);
+                va[0] &= m01;
+                va[1] &= m01;
+                va[2] &= m23;
+                va[3] &= m23;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_16816<BF16>(o[nt][mt], va, pb[nt][0], pb[nt][1]);
             }
 
             // stage consumed: hand it back to the producer for a later tile
@@ -535,48 +660,95 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         if (failed)
             break;
 
-        // ---- epilogue: final output (normalised) or a partial (m, l, o)
-        l_lo += __shfl_xor_sync(FULL, l_lo, 1);
-        l_lo += __shfl_xor_sync(FULL, l_lo, 2);
-        if constexpr (TWO) {
-            l_hi += __shfl_xor_sync(FULL, l_hi, 1);
-            l_hi += __shfl_xor_sync(FULL, l_hi, 2);
-        }
-        if (cs.dest < 0) {
-            const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
-            const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
-            if (g8 < rows) {
-                uint32_t *dst = reinterpret_cast<uint32_t *>(a.out + ((size_t)cs.seq * a.Hq + h0 + g8) * D);
-#pragma unroll
-                for (int j = 0; j < kNTiles; ++j)
-                    dst[j * 4 + c4] = pack2<BF16>(o[j][0] * inv_lo, o[j][1] * inv_lo);
+        // ---- epilogue: the fused append's cache store, then the outputs
+        if (has_new && new_slot >= 0) {
+            if (new_slot >= a.pool_slots) {
+                if (lane == 0)
+                    atomicOr(a.err, kErrSlot);
+            } else if (hg == 0 && lane < D / 4) {
+                const int64_t blk = new_slot / a.bs;
+                const int64_t row = new_slot - blk * a.bs;
+                const size_t dst = ((size_t)(blk * a.Hkv + kvh) * a.bs + row) * D;
+                reinterpret_cast<uint2 *>(a.k_cache + dst)[lane] = kn2;
+                reinterpret_cast<uint2 *>(a.v_cache + dst)[lane] = vn2;
             }
-            if (TWO && g8 + 8 < rows) {
-                uint32_t *dst = reinterpret_cast<uint32_t *>(a.out + ((size_t)cs.seq * a.Hq + h0 + g8 + 8) * D);
+        }
+        // per-head sums over the 16 token rows (lanes with the same c4)
 #pragma unroll
-                for (int j = 0; j < kNTiles; ++j)
-                    dst[j * 4 + c4] = pack2<BF16>(o[j][2] * inv_hi, o[j][3] * inv_hi);
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1)
+                    l_run[nt][j] += __shfl_xor_sync(FULL, l_run[nt][j], off);
+            }
+        }
+        // Accumulator 8x8 blocks are (d rows) x (head columns); movmatrix
+        // turns each into (head rows) x (d columns): lane (g8, c4) then owns
+        // head g8, d = 16*mt + 8*half + 2*c4 and the next one.
+        if (cs.dest < 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float inv0 = l_run[nt][0] > 0.f ? 1.f / l_run[nt][0] : 0.f;
+                const float inv1 = l_run[nt][1] > 0.f ? 1.f / l_run[nt][1] : 0.f;
+                const int head = nt * 8 + g8;
+                uint32_t *dst = reinterpret_cast<uint32_t *>(
+                    a.out + ((size_t)cs.seq * a.Hq + h0 + (head < rows ? head : 0)) * D);
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    const uint32_t b0 = movmatrix_trans(pack2<BF16>(o[nt][mt][0] * inv0, o[nt][mt][1] * inv1));
+                    const uint32_t b1 = movmatrix_trans(pack2<BF16>(o[nt][mt][2] * inv0, o[nt][mt][3] * inv1));
+                    if (head < rows) {
+                        dst[mt * 8 + c4] = b0;
+                        dst[mt * 8 + 4 + c4] = b1;
+                    }
+                }
             }
         } else {
-            for (int half = 0; half < (TWO ? 2 : 1); ++half) {
-                const int g = g8 + 8 * half;
-                if (g >= rows)
-                    continue;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int head = nt * 8 + g8;
                 size_t row;
                 if (a.mode == kModePartition)
-                    row = ((size_t)cs.seq * a.Hq + h0 + g) * a.S + cs.dest;
+                    row = ((size_t)cs.seq * a.Hq + h0 + head) * a.S + cs.dest;
                 else
-                    row = (size_t)cs.dest * kMaxRows + g;
-                float2 *dst = reinterpret_cast<float2 *>(a.part_o + row * D);
+                    row = (size_t)cs.dest * kMaxRows + head;
+                float *dst = a.part_o + row * D;
 #pragma unroll
-                for (int j = 0; j < kNTiles; ++j)
-                    dst[j * 4 + c4] = half ? make_float2(o[j][2], o[j][3]) : make_float2(o[j][0], o[j][1]);
-                if (c4 == 0) {
-                    a.part_m[row] = half ? m_hi : m_lo;
-                    a.part_l[row] = half ? l_hi : l_lo;
+                for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        // transpose the fp32 block as two 16-bit halves
+                        const uint32_t xb = __float_as_uint(o[nt][mt][2 * half]);
+                        const uint32_t yb = __float_as_uint(o[nt][mt][2 * half + 1]);
+                        const uint32_t hi = movmatrix_trans((xb >> 16) | (yb & 0xffff0000u));
+                        const uint32_t lo = movmatrix_trans((xb & 0xffffu) | (yb << 16));
+                        const float e0 = __uint_as_float((hi << 16) | (lo & 0xffffu));
+                        const float e1 = __uint_as_float((hi & 0xffff0000u) | (lo >> 16));
+                        if (head < rows)
+                            *reinterpret_cast<float2 *>(dst + mt * 16 + half * 8 + 2 * c4) = make_float2(e0, e1);
+                    }
+                }
+                // column state: lanes 0-3 hold heads 2*c4, 2*c4+1 of this n-tile
+                if (g8 == 0) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int hc = nt * 8 + 2 * c4 + j;
+                        if (hc < rows) {
+                            const size_t r = a.mode == kModePartition
+                                                 ? ((size_t)cs.seq * a.Hq + h0 + hc) * a.S + cs.dest
+                                                 : (size_t)cs.dest * kMaxRows + hc;
+                            a.part_m[r] = m_run[nt][j];
+                            a.part_l[r] = l_run[nt][j];
+                        }
+                    }
                 }
             }
         }
+        cw = nw;
+        cs = ns;
+        c_has = n_has;
+        cur = nxt;
     }
 
     if (failed) {
@@ -598,154 +770,287 @@ struct MergeArgs {
     const int32_t *prefix;   // balanced: tile prefix written by the decode kernel
     const float *part_o, *part_m, *part_l;
     int64_t mb;
-    int B, Hq, G, n_hg, npairs, bs, D;
+    int B, Hq, G, n_hg, npairs, bs;
+    int hpu;                 // query heads per decode unit (8 or 16)
     int mode, part_tiles, S, total_warps;
-    unsigned *err;
+};
+// Balanced mode: prefix[B + 1] holds an upper bound on the pieces per row;
+// partition mode: S is the bound.
+
+constexpr int kMergeThreads = 128;
+constexpr int kMergeChunk = 512;  // pieces staged in shared memory at a time
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
+    constexpr unsigned FULL = 0xffffffffu;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float x = __shfl_xor_sync(FULL, v, o);
+        v = is_max ? fmaxf(v, x) : v + x;
+    }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0)
+        red[warp] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int w = 1; w < kMergeThreads / 32; ++w)
+        r = is_max ? fmaxf(r, red[w]) : r + red[w];
+    __syncthreads();
+    return r;
+}
+
+// Where the pieces of one query head's split context are.
+struct MergeRow {
+    int seq, h, g;
+    long long count;   // pieces; <= 1 means nothing to merge
+    long long first;   // balanced: first warp
+    long long a0, T;   // balanced: flattened start of the pair, total tiles
 };
 
-constexpr int kMergeChunk = 64;
-
-// One CTA per (sequence, KV-head group): combine the partial results of the
-// pieces the context was split into.  M = max m_j, L = sum l_j 2^(m_j - M),
-// out = sum o_j 2^(m_j - M) / L.  Pieces with m = -inf weigh 0.
-template <bool BF16>
-__global__ void __launch_bounds__(256) lse_merge_kernel(const MergeArgs a) {
-    const int seq = blockIdx.x / a.npairs;
-    const int pair = blockIdx.x - seq * a.npairs;
-    const int kvh = pair / a.n_hg;
-    const int hg = pair - kvh * a.n_hg;
-    const int h0 = kvh * a.G + hg * kMaxRows;
-    const int rows = min(kMaxRows, a.G - hg * kMaxRows);
-
-    long long first = 0, count = 0;       // partition: j in [0, count)
-    long long a0 = 0, T = 0;              // balanced
+__device__ __forceinline__ MergeRow merge_row(const MergeArgs &a, long long row) {
+    MergeRow r;
+    r.seq = (int)(row / a.Hq);
+    r.h = (int)(row - (long long)r.seq * a.Hq);
+    const int kvh = r.h / a.G;
+    const int hl = r.h - kvh * a.G;
+    const int hg = hl / a.hpu;
+    r.g = hl - hg * a.hpu;
+    const int pair = kvh * a.n_hg + hg;
+    r.first = 0;
+    r.a0 = 0;
+    r.T = 1;
     if (a.mode == kModePartition) {
-        int c = a.context_lens[seq];
+        int c = a.context_lens[r.seq];
         const int64_t cap = a.mb * a.bs;
         c = c < 0 ? 0 : (c > cap ? (int)cap : c);
         const int nt = (c + kTileTokens - 1) / kTileTokens;
-        count = (nt + a.part_tiles - 1) / a.part_tiles;
-        if (count <= 1)
-            return;  // written directly by the decode kernel (or all-zero)
+        r.count = (nt + a.part_tiles - 1) / a.part_tiles;  // <= 1: written by the decode kernel
     } else {
-        const int nt = a.prefix[seq + 1] - a.prefix[seq];
-        if (nt == 0)
-            return;
-        T = (long long)a.prefix[a.B] * a.npairs;
-        a0 = (long long)a.prefix[seq] * a.npairs + (long long)pair * nt;
-        const long long b0 = a0 + nt;
-        const long long W = a.total_warps;
-        first = ((a0 + 1) * W + T - 1) / T - 1;        // warp holding index a0
-        const long long last = (b0 * W + T - 1) / T - 1;  // warp holding index b0 - 1
-        if (first == last)
-            return;  // the whole pair sat in one warp: already final
-        count = last - first + 1;
+        const int nt = a.prefix[r.seq + 1] - a.prefix[r.seq];
+        r.count = 0;
+        if (nt > 0) {
+            r.T = (long long)a.prefix[a.B] * a.npairs;
+            r.a0 = (long long)a.prefix[r.seq] * a.npairs + (long long)pair * nt;
+            const long long W = a.total_warps;
+            r.first = ((r.a0 + 1) * W + r.T - 1) / r.T - 1;                 // warp holding a0
+            const long long last = ((r.a0 + nt) * W + r.T - 1) / r.T - 1;  // warp holding a0+nt-1
+            r.count = last - r.first + 1;  // 1: the pair sat in one warp, already final
+        }
     }
+    return r;
+}
 
-    __shared__ float s_m[kMaxRows], s_inv[kMaxRows];
-    __shared__ float s_w[kMaxRows][kMergeChunk];
-    __shared__ long long s_row[kMergeChunk];  // partial row base (row index * 16 or per-head)
-    __shared__ int s_ok[kMergeChunk];
+// Partial row of piece k, or -1 (a warp whose range is empty).
+__device__ __forceinline__ long long merge_piece(const MergeArgs &a, const MergeRow &r, long long k) {
+    if (a.mode == kModePartition)
+        return ((long long)r.seq * a.Hq + r.h) * a.S + k;
+    const long long w = r.first + k;
+    if (r.T >= a.total_warps) {
+        // no warp has an empty range: the first piece is the first warp's
+        // last segment (slot 1), every later piece its warp's first (slot 0)
+        return (2 * w + (k == 0 ? 1 : 0)) * kMaxRows + r.g;
+    }
+    const long long lo = w * r.T / a.total_warps;
+    const long long hi = (w + 1) * r.T / a.total_warps;
+    if (lo >= hi)
+        return -1;
+    return (2 * w + (r.a0 < lo ? 0 : 1)) * kMaxRows + r.g;
+}
 
-    // row index of piece k for head row g
-    auto piece_row = [&](long long k, int g, bool &ok) -> long long {
-        ok = true;
-        if (a.mode == kModePartition)
-            return ((long long)seq * a.Hq + h0 + g) * a.S + k;
-        const long long w = first + k;
-        const long long lo = w * T / a.total_warps;
-        const long long hi = (w + 1) * T / a.total_warps;
-        if (lo >= hi) {
-            ok = false;
-            return 0;
+template <int D, bool BF16>
+__device__ __forceinline__ void store_row(const MergeArgs &a, const MergeRow &r, int c, const float *v,
+                                          int n) {
+    uint32_t *dst = reinterpret_cast<uint32_t *>(a.out + ((size_t)r.seq * a.Hq + r.h) * D + c);
+    for (int i = 0; i < n / 2; ++i)
+        dst[i] = pack2<BF16>(v[2 * i], v[2 * i + 1]);
+}
+
+constexpr int kWarpPieces = 64;  // rows with at most this many pieces: one warp each
+
+// One warp merges one row, kWarpPieces pieces at a time (rescaled online
+// across chunks): lanes hold two pieces' (row, m, l), the reductions are
+// shuffles, every lane owns D/32 consecutive outputs and issues its loads in
+// batches of eight.
+template <int D, bool BF16>
+__device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRow &r) {
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int VEC = D / 32;
+    const int lane = threadIdx.x & 31;
+    float M = -INFINITY, L = 0.f;
+    float acc[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i)
+        acc[i] = 0.f;
+    for (long long k0 = 0; k0 < r.count; k0 += kWarpPieces) {
+        long long rw[2];
+        float mw[2], lw[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const long long k = k0 + lane + 32 * j;
+            rw[j] = k < r.count ? merge_piece(a, r, k) : -1;
+            mw[j] = rw[j] >= 0 ? a.part_m[rw[j]] : -INFINITY;
+            lw[j] = rw[j] >= 0 ? a.part_l[rw[j]] : 0.f;
         }
-        const long long slot = 2 * w + (a0 < lo ? 0 : 1);
-        return slot * kMaxRows + g;
-    };
-
-    // pass 1: per-row max and normaliser
-    if (threadIdx.x < rows) {
-        const int g = threadIdx.x;
-        float M = -INFINITY;
-        for (long long k = 0; k < count; ++k) {
-            bool ok;
-            const long long r = piece_row(k, g, ok);
-            if (ok)
-                M = fmaxf(M, a.part_m[r]);
+        float cm = fmaxf(mw[0], mw[1]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
+        const float mnew = fmaxf(M, cm);
+        const float rescale = M == -INFINITY ? 0.f : exp2f(M - mnew);
+        float ww[2], lsum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            ww[j] = mw[j] == -INFINITY ? 0.f : exp2f(mw[j] - mnew);
+            lsum += ww[j] * lw[j];
         }
-        float Lsum = 0.f;
-        if (M != -INFINITY) {
-            for (long long k = 0; k < count; ++k) {
-                bool ok;
-                const long long r = piece_row(k, g, ok);
-                if (ok && a.part_m[r] != -INFINITY)
-                    Lsum += a.part_l[r] * exp2f(a.part_m[r] - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            lsum += __shfl_xor_sync(FULL, lsum, o);
+        L = L * rescale + lsum;
+        M = mnew;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i)
+            acc[i] *= rescale;
+        const int n = (int)min((long long)kWarpPieces, r.count - k0);
+#pragma unroll 8
+        for (int k = 0; k < n; ++k) {
+            const int j = k >> 5, src = k & 31;
+            const float w = __shfl_sync(FULL, j ? ww[1] : ww[0], src);
+            const long long rr = __shfl_sync(FULL, j ? rw[1] : rw[0], src);
+            if (w == 0.f)
+                continue;  // an empty piece: its (unwritten) row is never read
+            const float *p = a.part_o + rr * D + lane * VEC;
+            if constexpr (VEC == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(p);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2 *>(p);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
             }
         }
-        s_m[g] = M;
-        s_inv[g] = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i)
+        acc[i] *= inv;
+    store_row<D, BF16>(a, r, lane * VEC, acc, VEC);
+}
+
+// The whole CTA merges one row with many pieces: (row, m, l) staged in shared
+// memory in chunks (rescaled online across chunks), every thread owning one
+// 16-byte column slice and a stride of pieces.
+template <int D, bool BF16>
+__device__ __forceinline__ void merge_row_cta(const MergeArgs &a, const MergeRow &r, float *red,
+                                              long long *s_row, float *s_w, float *s_l, float4 *s_acc) {
+    constexpr int COLS = D / 4;
+    constexpr int GROUPS = kMergeThreads / COLS;
+    const int col = threadIdx.x % COLS;
+    const int grp = threadIdx.x / COLS;
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (long long k0 = 0; k0 < r.count; k0 += kMergeChunk) {
+        const int kn = (int)min((long long)kMergeChunk, r.count - k0);
+        float cmax = -INFINITY;
+        for (int i = threadIdx.x; i < kn; i += kMergeThreads) {
+            const long long rr = merge_piece(a, r, k0 + i);
+            const float m = rr >= 0 ? a.part_m[rr] : -INFINITY;
+            s_l[i] = rr >= 0 ? a.part_l[rr] : 0.f;
+            s_row[i] = rr;
+            s_w[i] = m;
+            cmax = fmaxf(cmax, m);
+        }
+        cmax = block_reduce(cmax, true, red);  // also orders the s_* writes
+        const float mnew = fmaxf(M, cmax);
+        const float rescale = M == -INFINITY ? 0.f : exp2f(M - mnew);
+        float lsum = 0.f;
+        for (int i = threadIdx.x; i < kn; i += kMergeThreads) {
+            const float m = s_w[i];
+            const float w = m == -INFINITY ? 0.f : exp2f(m - mnew);
+            s_w[i] = w;
+            lsum += w * s_l[i];
+        }
+        lsum = block_reduce(lsum, false, red);
+        L = L * rescale + lsum;
+        M = mnew;
+        acc.x *= rescale;
+        acc.y *= rescale;
+        acc.z *= rescale;
+        acc.w *= rescale;
+#pragma unroll 8
+        for (int i = grp; i < kn; i += GROUPS) {
+            const float w = s_w[i];
+            if (w == 0.f)
+                continue;  // an empty piece: its (unwritten) row is never read
+            const long long rr = s_row[i];
+            const float4 v = *reinterpret_cast<const float4 *>(a.part_o + rr * D + col * 4);
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+        }
+        __syncthreads();  // s_row / s_w / s_l are rewritten by the next chunk
+    }
+    s_acc[threadIdx.x] = acc;
+    __syncthreads();
+    if (threadIdx.x < COLS) {
+        float4 t = s_acc[threadIdx.x];
+#pragma unroll
+        for (int q = 1; q < GROUPS; ++q) {
+            const float4 u = s_acc[threadIdx.x + q * COLS];
+            t.x += u.x;
+            t.y += u.y;
+            t.z += u.z;
+            t.w += u.w;
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float v[4] = {t.x * inv, t.y * inv, t.z * inv, t.w * inv};
+        store_row<D, BF16>(a, r, threadIdx.x * 4, v, 4);
     }
     __syncthreads();
+}
 
-    // pass 2: weighted sum of the partial outputs, chunk by chunk.  Each
-    // thread owns up to kMaxPer pairs of consecutive d (rows <= 16, D <= 128,
-    // 256 threads).
-    constexpr int kMaxPer = 4;
-    const int D = a.D;
-    const int per_row = D / 2;
-    const int n_elem = rows * per_row;
-    float acc[kMaxPer][2];
-#pragma unroll
-    for (int e = 0; e < kMaxPer; ++e)
-        acc[e][0] = acc[e][1] = 0.f;
-    for (long long k0 = 0; k0 < count; k0 += kMergeChunk) {
-        const int kn = (int)min((long long)kMergeChunk, count - k0);
-        for (int i = threadIdx.x; i < rows * kn; i += blockDim.x) {
-            const int g = i / kn, k = i - g * kn;
-            bool ok;
-            const long long r = piece_row(k0 + k, g, ok);
-            float w = 0.f;
-            if (ok && s_m[g] != -INFINITY && a.part_m[r] != -INFINITY)
-                w = exp2f(a.part_m[r] - s_m[g]) * s_inv[g];
-            s_w[g][k] = w;
-            if (g == 0) {
-                s_row[k] = ok ? r : -1;
-                s_ok[k] = ok;
+// Combine the partial results (o_j unnormalised, m_j in the log2 domain, l_j)
+// of the pieces each query head's context was split into:
+//   M = max m_j,  L = sum l_j 2^(m_j - M),  out = sum o_j 2^(m_j - M) / L.
+// Pieces with m = -inf (no positions) weigh 0.  Each CTA takes four
+// consecutive (sequence, query head) rows, grid-stride: one warp per row when
+// every row has few pieces, else the four rows one after another with the
+// whole CTA.  The work is latency-bound (a few dependent round trips), so the
+// point is to keep many rows in flight.  Launched as a programmatic
+// dependent of the decode kernel, so its launch overlaps the decode tail.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergeArgs a) {
+    __shared__ float red[kMergeThreads / 32];
+    __shared__ long long s_row[kMergeChunk];
+    __shared__ float s_w[kMergeChunk];
+    __shared__ float s_l[kMergeChunk];
+    __shared__ float4 s_acc[kMergeThreads];
+    griddep_wait();
+    constexpr int ROWS = kMergeThreads / 32;
+    const int warp = threadIdx.x >> 5;
+    const long long rows_total = (long long)a.B * a.Hq;
+    const int bound = a.mode == kModePartition ? a.S : a.prefix[a.B + 1];
+    if (bound <= kWarpPieces) {
+        // few pieces per row: one warp per row, four rows per CTA
+        const long long groups = (rows_total + ROWS - 1) / ROWS;
+        for (long long grp = blockIdx.x; grp < groups; grp += gridDim.x) {
+            const long long row = grp * ROWS + warp;
+            if (row < rows_total) {
+                const MergeRow r = merge_row(a, row);
+                if (r.count > 1)
+                    merge_row_warp<D, BF16>(a, r);
             }
         }
-        __syncthreads();
-#pragma unroll
-        for (int e = 0; e < kMaxPer; ++e) {
-            const int idx = threadIdx.x + e * blockDim.x;
-            if (idx < n_elem) {
-                const int g = idx / per_row;
-                const int d = (idx - g * per_row) * 2;
-                float x0 = acc[e][0], x1 = acc[e][1];
-                for (int k = 0; k < kn; ++k) {
-                    if (!s_ok[k])
-                        continue;
-                    const float w = s_w[g][k];
-                    // rows of the other heads: +g*S (partition layout) or +g (slots)
-                    const long long r = a.mode == kModePartition ? s_row[k] + (long long)g * a.S
-                                                                 : s_row[k] + g;
-                    const float2 v = *reinterpret_cast<const float2 *>(a.part_o + r * D + d);
-                    x0 += w * v.x;
-                    x1 += w * v.y;
-                }
-                acc[e][0] = x0;
-                acc[e][1] = x1;
-            }
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int e = 0; e < kMaxPer; ++e) {
-        const int idx = threadIdx.x + e * blockDim.x;
-        if (idx < n_elem) {
-            const int g = idx / per_row;
-            const int d = (idx - g * per_row) * 2;
-            uint32_t *dst = reinterpret_cast<uint32_t *>(a.out + ((size_t)seq * a.Hq + h0 + g) * D + d);
-            *dst = pack2<BF16>(acc[e][0], acc[e][1]);
+    } else {
+        // many pieces per row: the whole CTA on one row
+        for (long long row = blockIdx.x; row < rows_total; row += gridDim.x) {
+            const MergeRow r = merge_row(a, row);
+            if (r.count > 1)
+                merge_row_cta<D, BF16>(a, r, red, s_row, s_w, s_l, s_acc);
         }
     }
 }
@@ -759,6 +1064,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint4 *__restrict__ k
                                                      int Hkv, int chunks, int bs, int64_t nb,
                                                      uint4 *__restrict__ k_cache,
                                                      uint4 *__restrict__ v_cache, unsigned *err) {
+    griddep_launch_dependents();
     const int64_t per_tok = (int64_t)Hkv * chunks;
     const int64_t total = T * per_tok;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;

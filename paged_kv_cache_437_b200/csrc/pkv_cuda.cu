@@ -8,7 +8,10 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <algorithm>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "decode.cuh"
 #include "pkv.h"
@@ -44,6 +47,17 @@ bool same_shape(const pkv_cache &a, const pkv_cache &b) {
            a.num_kv_heads == b.num_kv_heads && a.head_dim == b.head_dim;
 }
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Remember a failed runtime call for pkv_last_cuda_error().
+bool cuda_ok(cudaError_t e) {
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        return false;
+    }
+    return true;
+}
+
 unsigned *error_word() {
     static unsigned *ptr[64] = {};
     int dev = 0;
@@ -72,9 +86,40 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+bool make_pool_map_uncached(CUtensorMap *map, const pkv_cache &c);
+
+// Tensor maps are plain host encodings of (pointer, shape); a decode loop
+// over the same pool reuses them.
+bool make_pool_map(CUtensorMap *map, const pkv_cache &c) {
+    struct Entry {
+        void *data;
+        int dtype;
+        int64_t nb, bs, hkv, d;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const Entry &e : cache)
+            if (e.data == c.data && e.dtype == c.dtype && e.nb == c.num_blocks && e.bs == c.block_size &&
+                e.hkv == c.num_kv_heads && e.d == c.head_dim) {
+                *map = e.map;
+                return true;
+            }
+    }
+    if (!make_pool_map_uncached(map, c))
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 32)
+        cache.erase(cache.begin());
+    cache.push_back(Entry{c.data, (int)c.dtype, c.num_blocks, c.block_size, c.num_kv_heads, c.head_dim, *map});
+    return true;
+}
+
 // The pool viewed as a 2-D tensor: rows = NB * Hkv * bs, columns = D; one TMA
 // box = 16 rows x 64 columns (128 bytes per row), 128-byte swizzle.
-bool make_pool_map(CUtensorMap *map, const pkv_cache &c) {
+bool make_pool_map_uncached(CUtensorMap *map, const pkv_cache &c) {
     auto fn = encode_fn();
     if (!fn)
         return false;
@@ -102,39 +147,116 @@ struct Plan {
     int S = 0;
     int smem = 0;
     int Hkv = 0, G = 0, n_hg = 0, npairs = 0;
+    int nt = 1, hpu = 8;  // MMA column tiles and query heads per unit
 };
 
 using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
-DecodeKernel pick_decode(int D, bool bf16, bool two) {
-#define PKV_PICK(DD, BB, TT) \
-    if (D == DD && bf16 == BB && two == TT) return paged_decode_kernel<DD, BB, TT>;
-    PKV_PICK(64, false, false)
-    PKV_PICK(64, false, true)
-    PKV_PICK(64, true, false)
-    PKV_PICK(64, true, true)
-    PKV_PICK(128, false, false)
-    PKV_PICK(128, false, true)
-    PKV_PICK(128, true, false)
-    PKV_PICK(128, true, true)
+// NT = number of 8-head MMA column tiles per unit: 1 for G <= 8, else 2.
+DecodeKernel pick_decode(int D, bool bf16, int nt) {
+#define PKV_PICK(DD, BB, NN) \
+    if (D == DD && bf16 == BB && nt == NN) return paged_decode_kernel<DD, BB, NN>;
+    PKV_PICK(64, false, 1)
+    PKV_PICK(64, false, 2)
+    PKV_PICK(64, true, 1)
+    PKV_PICK(64, true, 2)
+    PKV_PICK(128, false, 1)
+    PKV_PICK(128, false, 2)
+    PKV_PICK(128, true, 1)
+    PKV_PICK(128, true, 2)
 #undef PKV_PICK
     return nullptr;
 }
 
 int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel in the stream is still running; it calls
+// griddepcontrol.wait before reading anything that kernel may have written.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Decide schedule, CTA shape and grid.  PKV_ERR_INVALID if the shape cannot
 // be run (shared memory), PKV_ERR_CUDA if the device cannot be queried.
+pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
+                              int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch);
+
+// Plans depend only on the shape, the device and two tuning variables; they
+// are cached so that a steady decode loop pays no occupancy queries.
+struct PlanKey {
+    int dev, warps_env, stages_env;
+    int64_t B, Hq, Hkv, D, max_ctx;
+    int32_t partition;
+    bool ws, bf16, launch;
+    bool operator==(const PlanKey &o) const {
+        return dev == o.dev && warps_env == o.warps_env && stages_env == o.stages_env && B == o.B &&
+               Hq == o.Hq && Hkv == o.Hkv && D == o.D && max_ctx == o.max_ctx &&
+               partition == o.partition && ws == o.ws && bf16 == o.bf16 && launch == o.launch;
+    }
+};
+
 pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
-               int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch) {
+                     int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch) {
+    static std::mutex mu;
+    static std::vector<std::pair<PlanKey, Plan>> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const PlanKey key{dev, env_int("PKV_WARPS", 0), env_int("PKV_STAGES", 0), B, Hq, Hkv, D, max_ctx,
+                      partition_tokens, have_workspace, bf16, for_launch};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (auto &e : cache)
+            if (e.first == key) {
+                p = e.second;
+                return PKV_OK;
+            }
+    }
+    pkv_status st = make_plan_uncached(p, B, Hq, Hkv, D, max_ctx, partition_tokens, have_workspace, bf16,
+                                       for_launch);
+    if (st == PKV_OK) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (cache.size() >= 64)
+            cache.erase(cache.begin());
+        cache.emplace_back(key, p);
+    }
+    return st;
+}
+
+pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
+                              int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch) {
     p.Hkv = (int)Hkv;
     p.G = (int)(Hq / Hkv);
-    p.n_hg = (p.G + kMaxRows - 1) / kMaxRows;
+    p.nt = p.G > 8 ? 2 : 1;
+    p.hpu = 8 * p.nt;
+    p.n_hg = (p.G + p.hpu - 1) / p.hpu;
     p.npairs = (int)Hkv * p.n_hg;
-    p.warps = env_int("PKV_WARPS", 4);
-    p.stages = env_int("PKV_STAGES", D == 64 ? 6 : 3);
+    // CTA shape, from measurements on B200 (two 8 KB stages per warp):
+    //  * fixed partitions are equal-sized units whose makespan is
+    //    ceil(units / warps) units: as many resident warps as fit (7 per CTA,
+    //    two CTAs per SM);
+    //  * large batches (>= 128 sequences, continuous-batching mixes) switch
+    //    units often and hide that latency best with 12 warps per SM (two
+    //    6-warp CTAs);
+    //  * otherwise one 8-warp CTA per SM.
+    const int dflt_warps = partition_tokens > 0 ? 7 : (B >= 128 ? 6 : 8);
+    p.warps = env_int("PKV_WARPS", dflt_warps);
+    p.stages = env_int("PKV_STAGES", 2);
     if (p.warps < 1 || p.warps > 8)
-        p.warps = 4;
+        p.warps = 8;
     if (p.stages < 2 || p.stages > 16)
         p.stages = 3;
     if (partition_tokens > 0) {
@@ -169,10 +291,13 @@ pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int
         return PKV_ERR_CUDA;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int per_sm = 1;
-    DecodeKernel k = pick_decode((int)D, bf16, p.G > 8);
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt);
     if (!k)
         return PKV_ERR_INVALID;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) != cudaSuccess)
+    // The attribute is per-kernel state shared by every cached plan: set the
+    // ceiling, never a plan's own size (a smaller plan would otherwise lower
+    // it under a larger one).  It only permits; occupancy uses p.smem.
+    if (!cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta)))
         return PKV_ERR_CUDA;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, p.warps * 32, p.smem) !=
             cudaSuccess ||
@@ -199,7 +324,7 @@ pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int
 
 // Workspace layout.
 //  partition: part_o [B][Hq][S][D] f32 | part_m [B][Hq][S] f32 | part_l [B][Hq][S] f32
-//  balanced:  prefix [B+1] i32 (256-aligned) | part_m [2W][16] | part_l [2W][16] | part_o [2W][16][D]
+//  balanced:  prefix [B+1] i32 + pieces bound (256-aligned) | part_m [2W][16] | part_l [2W][16] | part_o [2W][16][D]
 //             with W = the largest warp count a launch may use.
 struct WsLayout {
     size_t prefix = 0, m = 0, l = 0, o = 0, total = 0;
@@ -218,7 +343,7 @@ WsLayout ws_layout(const Plan &p, int64_t B, int64_t Hq, int64_t D, int64_t max_
     } else if (p.mode == kModeBalanced) {
         const size_t slots = (size_t)2 * max_warps;
         w.prefix = 0;
-        w.m = align256((size_t)(B + 1) * 4);
+        w.m = align256((size_t)(B + 2) * 4);
         w.l = align256(w.m + slots * kMaxRows * 4);
         w.o = align256(w.l + slots * kMaxRows * 4);
         w.total = align256(w.o + slots * kMaxRows * D * 4);
@@ -260,7 +385,7 @@ pkv_status pkv_append(const void *k_new, const void *v_new, const int64_t *slot_
         num_tokens, (int)k_cache.num_kv_heads, chunks, (int)k_cache.block_size,
         k_cache.num_blocks, static_cast<uint4 *>(k_cache.data), static_cast<uint4 *>(v_cache.data),
         err);
-    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_ok(cudaGetLastError()) ? PKV_OK : PKV_ERR_CUDA;
 }
 
 size_t pkv_decode_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
@@ -280,11 +405,20 @@ size_t pkv_decode_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t
     return ws_layout(p, num_seqs, num_q_heads, head_dim, p.max_total_warps).total;
 }
 
-pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_heads,
-                                pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
-                                int64_t max_blocks_per_seq, const int32_t *context_lens,
-                                float scale, void *out, void *workspace, size_t workspace_bytes,
-                                int32_t partition_tokens, pkv_stream stream) {
+}  // extern "C"
+
+namespace {
+
+struct FusedAppend {
+    const void *k_new, *v_new;
+    const int64_t *slots;
+};
+
+pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv_cache k_cache,
+                       pkv_cache v_cache, const int32_t *block_tables, int64_t max_blocks_per_seq,
+                       const int32_t *context_lens, float scale, void *out, void *workspace,
+                       size_t workspace_bytes, int32_t partition_tokens, pkv_stream stream,
+                       const FusedAppend *fa) {
     if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0)
         return PKV_ERR_INVALID;
     if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
@@ -368,10 +502,16 @@ pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_h
     a.err = err;
     a.wait_limit_ns = g_wait_limit_ns;
     a.inject_no_issue = g_inject_no_issue;
+    a.k_new = fa ? static_cast<const uint16_t *>(fa->k_new) : nullptr;
+    a.v_new = fa ? static_cast<const uint16_t *>(fa->v_new) : nullptr;
+    a.slots = fa ? fa->slots : nullptr;
+    a.k_cache = static_cast<uint16_t *>(k_cache.data);
+    a.v_cache = static_cast<uint16_t *>(v_cache.data);
+    a.pool_slots = k_cache.num_blocks * bs;
 
-    DecodeKernel k = pick_decode((int)D, bf16, p.G > 8);
-    k<<<p.ctas, p.warps * 32, p.smem, (cudaStream_t)stream>>>(tmK, tmV, a);
-    if (cudaGetLastError() != cudaSuccess)
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt);
+    if (!cuda_ok(launch_dependent(k, dim3(p.ctas), dim3(p.warps * 32), p.smem, (cudaStream_t)stream, tmK,
+                                  tmV, a)))
         return PKV_ERR_CUDA;
 
     const bool merge = (p.mode == kModeBalanced) || (p.mode == kModePartition && p.S > 1);
@@ -390,25 +530,68 @@ pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_h
         m.n_hg = a.n_hg;
         m.npairs = a.npairs;
         m.bs = a.bs;
-        m.D = (int)D;
+        m.hpu = p.hpu;
         m.mode = p.mode;
         m.part_tiles = p.part_tiles;
         m.S = p.S;
         m.total_warps = p.total_warps;
-        m.err = err;
-        const int64_t grid = num_seqs * p.npairs;
-        if (bf16)
-            lse_merge_kernel<true><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(m);
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        // enough CTAs for one row each when rows have many pieces; with few
+        // pieces a CTA takes four rows and the rest exit at once
+        const unsigned grid = (unsigned)std::min<int64_t>(num_seqs * num_q_heads, (int64_t)sms * 8);
+        cudaError_t e;
+        if (D == 128)
+            e = bf16 ? launch_dependent(lse_merge_kernel<128, true>, dim3(grid), dim3(kMergeThreads), 0,
+                                        (cudaStream_t)stream, m)
+                     : launch_dependent(lse_merge_kernel<128, false>, dim3(grid), dim3(kMergeThreads), 0,
+                                        (cudaStream_t)stream, m);
         else
-            lse_merge_kernel<false><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(m);
-        if (cudaGetLastError() != cudaSuccess)
+            e = bf16 ? launch_dependent(lse_merge_kernel<64, true>, dim3(grid), dim3(kMergeThreads), 0,
+                                        (cudaStream_t)stream, m)
+                     : launch_dependent(lse_merge_kernel<64, false>, dim3(grid), dim3(kMergeThreads), 0,
+                                        (cudaStream_t)stream, m);
+        if (!cuda_ok(e))
             return PKV_ERR_CUDA;
     }
     return PKV_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_decode_attention(const void *q, int64_t num_seqs, int64_t num_q_heads,
+                                pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+                                int64_t max_blocks_per_seq, const int32_t *context_lens,
+                                float scale, void *out, void *workspace, size_t workspace_bytes,
+                                int32_t partition_tokens, pkv_stream stream) {
+    return decode_impl(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                       context_lens, scale, out, workspace, workspace_bytes, partition_tokens, stream,
+                       nullptr);
+}
+
+pkv_status pkv_append_decode_attention(const void *k_new, const void *v_new,
+                                       const int64_t *slot_mapping, const void *q, int64_t num_seqs,
+                                       int64_t num_q_heads, pkv_cache k_cache, pkv_cache v_cache,
+                                       const int32_t *block_tables, int64_t max_blocks_per_seq,
+                                       const int32_t *context_lens, float scale, void *out,
+                                       void *workspace, size_t workspace_bytes,
+                                       int32_t partition_tokens, pkv_stream stream) {
+    if (num_seqs > 0 && (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new) ||
+                         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u)))
+        return PKV_ERR_INVALID;
+    const FusedAppend fa{k_new, v_new, slot_mapping};
+    return decode_impl(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                       context_lens, scale, out, workspace, workspace_bytes, partition_tokens, stream,
+                       &fa);
+}
+
+const char *pkv_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
 pkv_status pkv_get_last_error(void) {
-    if (cudaDeviceSynchronize() != cudaSuccess)
+    if (!cuda_ok(cudaDeviceSynchronize()))
         return PKV_ERR_CUDA;
     unsigned *err = error_word();
     if (!err)

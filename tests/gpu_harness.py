@@ -98,6 +98,15 @@ class GpuStep:
         pkv.pkv_decode_attention(self.q, self.kc, self.vc, self.tables, self.lens, self.w.scale, self.out,
                                  workspace, partition, stream)
 
+    def run_fused(self, partition: int = pkv.PKV_PARTITION_AUTO):
+        ws = workspace_for(self.w, partition)
+        pkv.pkv_append_decode_attention(self.kn, self.vn, self.slots, self.q, self.kc, self.vc, self.tables,
+                                        self.lens, self.w.scale, self.out, ws, partition)
+        torch.cuda.synchronize()
+        st = pkv.pkv_get_last_error()
+        assert st == pkv.PKV_OK, pkv.pkv_status_string(st)
+        return self.out
+
     def run(self, partition: int = pkv.PKV_PARTITION_AUTO):
         ws = workspace_for(self.w, partition)
         self.append()

@@ -48,6 +48,21 @@ def test_small_shapes_elementwise(small_case, mode):
     gh.assert_close(gh.to_f64(out), ref, w.spec.dtype, f"{w.spec.name} mode {mode}")
 
 
+@pytest.mark.parametrize("mode", [pkv.PKV_PARTITION_NONE, pkv.PKV_PARTITION_AUTO, 512, 16], ids=lambda m: f"part{m}")
+def test_fused_append_decode_small_shapes(small_case, mode):
+    """pkv_append_decode_attention: same pool and the same output bits as
+    pkv_append followed by pkv_decode_attention, and within tolerance of the oracle."""
+    w, kc, vc, slots, ref, k_ref, v_ref = small_case
+    fused = gh.GpuStep(w, kc, vc, slots)
+    out_f = fused.run_fused(mode).clone()
+    assert np.array_equal(gh.host_bits(fused.kc), k_ref), "fused: appended K pool differs"
+    assert np.array_equal(gh.host_bits(fused.vc), v_ref), "fused: appended V pool differs"
+    gh.assert_close(gh.to_f64(out_f), ref, w.spec.dtype, f"fused {w.spec.name} mode {mode}")
+    sep = gh.GpuStep(w, kc, vc, slots)
+    out_s = sep.run(mode)
+    assert np.array_equal(gh.host_bits(out_f), gh.host_bits(out_s)), "fused and separate calls differ"
+
+
 FULL_MODES = {
     "tiny": [pkv.PKV_PARTITION_AUTO, pkv.PKV_PARTITION_NONE, 512],
     "llama13b": [pkv.PKV_PARTITION_AUTO],
@@ -64,10 +79,10 @@ def test_named_workload_full_size(name):
     pairs = None if name == "tiny" else gh.sample_pairs(w, 64)
     ref, k_ref, v_ref = gh.oracle_step(w, kc, vc, slots, pairs=pairs)
     step = gh.GpuStep(w, kc, vc, slots)
-    for mode in FULL_MODES[name]:
+    for mode, fused in [(m, f) for m in FULL_MODES[name] for f in (False, True)]:
         step.kc.copy_(gh.dev(kc, w.spec.dtype))
         step.vc.copy_(gh.dev(vc, w.spec.dtype))
-        out = step.run(mode)
+        out = step.run_fused(mode) if fused else step.run(mode)
         assert np.array_equal(gh.host_bits(step.kc), k_ref), f"{name}: appended K pool differs"
         assert np.array_equal(gh.host_bits(step.vc), v_ref), f"{name}: appended V pool differs"
         got = gh.to_f64(out)
@@ -75,4 +90,5 @@ def test_named_workload_full_size(name):
         if pairs is not None:
             got = got[pairs[:, 0], pairs[:, 1]]
         err = gh.assert_close(got, ref, w.spec.dtype, f"{name} mode {mode}")
-        print(f"{name} mode {mode}: {len(ref) if pairs is not None else ref.size} compared, max |err| {err:.3e}")
+        print(f"{name} mode {mode} fused {fused}: {len(ref) if pairs is not None else ref.size} compared, "
+              f"max |err| {err:.3e}")
