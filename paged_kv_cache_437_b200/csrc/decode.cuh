@@ -459,70 +459,56 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
     int consumed = 0;
     bool failed = false;
 
-    // Per-unit inputs -- the query fragments and, for a fused append, the new
-    // token's row and slot -- are loaded one unit ahead: the loads for unit
-    // u+1 are issued when unit u starts and first used when u+1 starts.
-    struct UnitIn {
-        uint32_t qb[NT][kMT][2];  // Q^T as the B operand (k = head dim, n = query head)
-        bool has_new;             // this unit holds its sequence's last position
-        int64_t slot;
-        uint2 kn, vn;
-    };
-    auto load_unit = [&](const Seg &u, UnitIn &in) {
-        const int kvh_u = u.pair / a.n_hg;
-        const int hg_u = u.pair - kvh_u * a.n_hg;
-        const int h0_u = kvh_u * a.G + hg_u * HPU;
-        const int rows_u = min(HPU, a.G - hg_u * HPU);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int head = nt * 8 + g8;
-            const bool valid = head < rows_u;
-            const uint32_t *qr = reinterpret_cast<const uint32_t *>(
-                a.q + ((size_t)u.seq * a.Hq + h0_u + (valid ? head : 0)) * D);
-#pragma unroll
-            for (int ks = 0; ks < kMT; ++ks) {
-                in.qb[nt][ks][0] = valid ? __ldg(qr + ks * 8 + c4) : 0u;
-                in.qb[nt][ks][1] = valid ? __ldg(qr + ks * 8 + 4 + c4) : 0u;
-            }
-        }
-        in.has_new = a.k_new != nullptr && u.t1 > u.t0 && u.t1 * kTileTokens >= u.ctx;
-        in.slot = -1;
-        in.kn = in.vn = make_uint2(0, 0);
-        if (in.has_new) {
-            in.slot = __ldg(a.slots + u.seq);
-            if (lane < D / 4) {
-                const size_t src = ((size_t)u.seq * a.Hkv + kvh_u) * D;
-                in.kn = __ldg(reinterpret_cast<const uint2 *>(a.k_new + src) + lane);
-                in.vn = __ldg(reinterpret_cast<const uint2 *>(a.v_new + src) + lane);
-            }
-        }
-    };
-
-    bool c_has = walker_next(cw, cs, a, prefix, ctxs, gw);
-    UnitIn cur;
-    if (c_has)
-        load_unit(cs, cur);
-    while (!failed && c_has) {
+    while (!failed && walker_next(cw, cs, a, prefix, ctxs, gw)) {
         const int kvh = cs.pair / a.n_hg;
         const int hg = cs.pair - kvh * a.n_hg;
         const int h0 = kvh * a.G + hg * HPU;
         const int rows = min(HPU, a.G - hg * HPU);
 
-        // issue the next unit's loads now; they land while this unit runs
-        Walker nw = cw;
-        Seg ns;
-        const bool n_has = walker_next(nw, ns, a, prefix, ctxs, gw);
-        UnitIn nxt;
-        if (n_has)
-            load_unit(ns, nxt);
+        // Q^T as the B operand (k = head dim, n = query head)
+        uint32_t qb[NT][kMT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = nt * 8 + g8;
+            const bool valid = head < rows;
+            const uint32_t *qr =
+                reinterpret_cast<const uint32_t *>(a.q + ((size_t)cs.seq * a.Hq + h0 + (valid ? head : 0)) * D);
+#pragma unroll
+            for (int ks = 0; ks < kMT; ++ks) {
+                qb[nt][ks][0] = valid ? __ldg(qr + ks * 8 + c4) : 0u;
+                qb[nt][ks][1] = valid ? __ldg(qr + ks * 8 + 4 + c4) : 0u;
+            }
+        }
 
-        // Fused append: the unit that holds the sequence's last position
-        // patches the new K/V row into its shared-memory tile at the last
-        // tile and stores it to its cache slot in the epilogue (once per KV
-        // head: head group 0).
-        const bool has_new = cur.has_new;
-        const int64_t new_slot = cur.slot;
-        const uint2 kn2 = cur.kn, vn2 = cur.vn;
+        {
+            // pull the next unit's query rows into L2 while this one runs
+            Walker nw = cw;
+            Seg ns;
+            if (walker_next(nw, ns, a, prefix, ctxs, gw)) {
+                const int nk = ns.pair / a.n_hg;
+                const int nh = ns.pair - nk * a.n_hg;
+                const int nrows = min(HPU, a.G - nh * HPU);
+                const char *base = reinterpret_cast<const char *>(
+                    a.q + ((size_t)ns.seq * a.Hq + nk * a.G + nh * HPU) * D);
+                if (lane * 128 < nrows * D * 2)
+                    prefetch_l2(base + lane * 128);
+            }
+        }
+
+        // Fused append: this unit holds its sequence's last position.  The
+        // new token's row (one 8-byte piece per lane) and slot are loaded here,
+        // together with Q, and first used at the last tile.
+        const bool has_new = a.k_new != nullptr && cs.t1 > cs.t0 && cs.t1 * kTileTokens >= cs.ctx;
+        int64_t new_slot = -1;
+        uint2 kn2 = make_uint2(0, 0), vn2 = make_uint2(0, 0);
+        if (has_new) {
+            new_slot = __ldg(a.slots + cs.seq);
+            if (lane < D / 4) {
+                const size_t src = ((size_t)cs.seq * a.Hkv + kvh) * D;
+                kn2 = __ldg(reinterpret_cast<const uint2 *>(a.k_new + src) + lane);
+                vn2 = __ldg(reinterpret_cast<const uint2 *>(a.v_new + src) + lane);
+            }
+        }
 
         float o[NT][kMT][4];
         float m_run[NT][2], l_run[NT][2];
@@ -549,6 +535,19 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const uint32_t kb = ring_base + stage * 2 * kTile;
             const uint32_t vb = kb + kTile;
             const int nvalid = min(kTileTokens, cs.ctx - t * kTileTokens);
+            if (has_new && t == cs.t1 - 1 && new_slot >= 0) {
+                if (new_slot >= a.pool_slots) {
+                    if (lane == 0)
+                        atomicOr(a.err, kErrSlot);
+                } else if (hg == 0 && lane < D / 4) {
+                    // the append proper: the new row to its cache slot
+                    const int64_t blk = new_slot / a.bs;
+                    const int64_t row = new_slot - blk * a.bs;
+                    const size_t dst = ((size_t)(blk * a.Hkv + kvh) * a.bs + row) * D;
+                    reinterpret_cast<uint2 *>(a.k_cache + dst)[lane] = kn2;
+                    reinterpret_cast<uint2 *>(a.v_cache + dst)[lane] = vn2;
+                }
+            }
             if (has_new && t == cs.t1 - 1 && new_slot >= 0 && new_slot < a.pool_slots) {
                 // the new token's row of this tile, in the 128-byte swizzle
                 const int r = cs.ctx - 1 - t * kTileTokens;
@@ -580,7 +579,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 ldmatrix_x4(addr, ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
-                    mma_16816<BF16>(sc[nt], ka, cur.qb[nt][ks][0], cur.qb[nt][ks][1]);
+                    mma_16816<BF16>(sc[nt], ka, qb[nt][ks][0], qb[nt][ks][1]);
             }
 
             // online softmax per query head (one column of S^T), log2 domain;
@@ -660,20 +659,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         if (failed)
             break;
 
-        // ---- epilogue: the fused append's cache store, then the outputs
-        if (has_new && new_slot >= 0) {
-            if (new_slot >= a.pool_slots) {
-                if (lane == 0)
-                    atomicOr(a.err, kErrSlot);
-            } else if (hg == 0 && lane < D / 4) {
-                const int64_t blk = new_slot / a.bs;
-                const int64_t row = new_slot - blk * a.bs;
-                const size_t dst = ((size_t)(blk * a.Hkv + kvh) * a.bs + row) * D;
-                reinterpret_cast<uint2 *>(a.k_cache + dst)[lane] = kn2;
-                reinterpret_cast<uint2 *>(a.v_cache + dst)[lane] = vn2;
-            }
-        }
-        // per-head sums over the 16 token rows (lanes with the same c4)
+        // ---- epilogue: per-head sums over the 16 token rows (lanes with the same c4)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -745,10 +731,6 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 }
             }
         }
-        cw = nw;
-        cs = ns;
-        c_has = n_has;
-        cur = nxt;
     }
 
     if (failed) {

@@ -245,14 +245,11 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
     p.n_hg = (p.G + p.hpu - 1) / p.hpu;
     p.npairs = (int)Hkv * p.n_hg;
     // CTA shape, from measurements on B200 (two 8 KB stages per warp):
-    //  * fixed partitions are equal-sized units whose makespan is
-    //    ceil(units / warps) units: as many resident warps as fit (7 per CTA,
-    //    two CTAs per SM);
     //  * large batches (>= 128 sequences, continuous-batching mixes) switch
     //    units often and hide that latency best with 12 warps per SM (two
     //    6-warp CTAs);
     //  * otherwise one 8-warp CTA per SM.
-    const int dflt_warps = partition_tokens > 0 ? 7 : (B >= 128 ? 6 : 8);
+    const int dflt_warps = (partition_tokens <= 0 && B >= 128) ? 6 : 8;
     p.warps = env_int("PKV_WARPS", dflt_warps);
     p.stages = env_int("PKV_STAGES", 2);
     if (p.warps < 1 || p.warps > 8)
@@ -315,6 +312,14 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
             units = B * p.npairs * p.S;
         else
             units = ceil_div64(B * p.npairs * tiles_upper, 4);  // >= ~4 tiles per warp
+        if (p.mode == kModePartition) {
+            // equal-sized units taken round-robin: the makespan is
+            // ceil(units / warps) units; keep the smallest makespan the grid
+            // allows with the fewest warps (less contention for the same time)
+            const int64_t max_w = max_ctas * p.warps;
+            const int64_t rounds = ceil_div64(units, max_w);
+            units = ceil_div64(units, rounds);
+        }
         want = std::min<int64_t>(max_ctas, std::max<int64_t>(1, ceil_div64(units, p.warps)));
     }
     p.ctas = (int)want;
