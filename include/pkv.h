@@ -98,6 +98,17 @@ pkv_status pkv_append(const void *k_new, const void *v_new,
                       pkv_cache k_cache, pkv_cache v_cache, pkv_stream stream);
 
 /* --------------------------------------------------------------------------
+ * pkv_copy_blocks -- device side of copy-on-write: for each (src, dst) pair
+ * of pairs (device int32 [n][2]) copy the whole physical block src to dst in
+ * both pools (all KV heads and rows: Hkv * bs * D values each).  The dst
+ * blocks must be distinct and no dst may also be a src (the pairs from the
+ * copy-on-write appends satisfy this), so the copies are independent.  An id
+ * outside [0, NB) is skipped and flagged (PKV_ERR_DEVICE_CHECK).
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_copy_blocks(pkv_cache k_cache, pkv_cache v_cache, const int32_t *pairs,
+                           int64_t num_pairs, pkv_stream stream);
+
+/* --------------------------------------------------------------------------
  * pkv_decode_attention -- one decode step of attention over the paged cache.
  * [KVB] "The KV cache": attention needs the keys and values of all prior
  * positions; decode generates one token at a time.  [KVB] "PagedAttention and
@@ -260,6 +271,25 @@ pkv_status pkv_seq_append_slot(void *h, int32_t seq, int64_t *slot_out);
 /* pkv_seq_append_slot for n sequences at once, all or nothing: on an error
  * (including OOM for the batch as a whole) no sequence changes. */
 pkv_status pkv_seq_append_slots(void *h, const int32_t *seqs, int32_t n, int64_t *slots_out);
+/* Copy-on-write sharing (the plain reading of sharing pages between
+ * requests that keep appending): a fork may share the parent's first
+ * num_tokens positions including a partly filled last block (each shared
+ * block gets one more reference); the child starts with context length
+ * num_tokens. */
+pkv_status pkv_seq_fork_tokens(void *h, int32_t parent, int64_t num_tokens, int32_t *child_out);
+/* pkv_seq_append_slot, except that an append into a shared block first gives
+ * the sequence a private copy: a fresh block replaces the shared one in its
+ * table (the shared block loses one reference) and (*copy_src, *copy_dst)
+ * name the block copy the caller must make on the device (pkv_copy_blocks)
+ * before writing the token; both are -1 when no copy is needed.  OOM leaves
+ * everything unchanged. */
+pkv_status pkv_seq_append_slot_cow(void *h, int32_t seq, int64_t *slot_out, int32_t *copy_src,
+                                   int32_t *copy_dst);
+/* Batch form, all or nothing: copies_out[2*k], copies_out[2*k+1] receive the
+ * k-th (src, dst) copy, *n_copies_out their number (at most n). */
+pkv_status pkv_seq_append_slots_cow(void *h, const int32_t *seqs, int32_t n, int64_t *slots_out,
+                                    int32_t *copies_out, int32_t *n_copies_out);
+
 /* Drop the sequence: every block loses one reference; blocks reaching 0
  * return to the free list.  The id may be reused by a later create/fork. */
 pkv_status pkv_seq_free(void *h, int32_t seq);

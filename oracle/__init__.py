@@ -58,6 +58,8 @@ def _bind(lib):
         vp, i64, vp]
     lib.oracle_lse_merge.restype = ctypes.c_int
     lib.oracle_lse_merge.argtypes = [i64, vp, vp, vp, i64, vp]
+    lib.oracle_copy_blocks.restype = ctypes.c_int
+    lib.oracle_copy_blocks.argtypes = [vp, i64, i64, vp, i64]
     lib.oracle_mark_slots.restype = ctypes.c_int
     lib.oracle_mark_slots.argtypes = [vp, i64, i64, vp, i64, i64, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -204,6 +206,17 @@ def slot_mask(block_tables, lens, block_size: int, num_blocks: int, lib=None) ->
     if rc != 0:
         raise ValueError("oracle_mark_slots: table entry out of range")
     return mask.astype(bool)
+
+
+def copy_blocks(cache: np.ndarray, pairs, lib=None) -> None:
+    """In-place whole-block copies src -> dst of a [NB][Hkv][bs][D] pool, in order."""
+    lib = lib or load()
+    assert cache.flags.c_contiguous
+    nb = cache.shape[0]
+    pr = np.ascontiguousarray(pairs, dtype=np.int32).reshape(-1, 2)
+    rc = lib.oracle_copy_blocks(_p(cache.view(np.uint16)), nb, int(np.prod(cache.shape[1:])), _p(pr), len(pr))
+    if rc != 0:
+        raise ValueError("oracle_copy_blocks: block id out of range")
 
 
 def num_threads(lib=None) -> int:

@@ -345,3 +345,25 @@ int oracle_mark_slots(const int32_t *block_tables, int64_t num_seqs,
     }
     return 0;
 }
+
+/*
+ * Copy-on-write support: copy whole physical blocks (all KV heads, all rows)
+ * src -> dst for each (src, dst) pair, in order.  A block is
+ * kv_heads * block_size * head_dim 16-bit values, contiguous in the pool.
+ * Sharing pages between requests with a common prefix is the pages' idea
+ * (adilsher.pro post, "The Elegant Fix: Paged Attention"); a writer of a
+ * shared page gets a private copy first (the plain reading of sharing with
+ * appends).  Returns -1 if an id is outside [0, num_blocks).
+ */
+int oracle_copy_blocks(uint16_t *cache, int64_t num_blocks, int64_t block_elems,
+                       const int32_t *pairs, int64_t num_pairs)
+{
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks)
+            return -1;
+        memmove(cache + dst * block_elems, cache + src * block_elems,
+                (size_t)block_elems * sizeof(uint16_t));
+    }
+    return 0;
+}

@@ -72,6 +72,11 @@ def _load():
         "pkv_seq_append_slot": (ctypes.c_int, [_c_vp, _c_i32, ctypes.POINTER(_c_i64)]),
         "pkv_seq_append_slots": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp]),
         "pkv_seq_free": (ctypes.c_int, [_c_vp, _c_i32]),
+        "pkv_seq_fork_tokens": (ctypes.c_int, [_c_vp, _c_i32, _c_i64, ctypes.POINTER(_c_i32)]),
+        "pkv_seq_append_slot_cow": (ctypes.c_int, [_c_vp, _c_i32, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i32),
+                                                   ctypes.POINTER(_c_i32)]),
+        "pkv_seq_append_slots_cow": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp, ctypes.POINTER(_c_i32)]),
+        "pkv_copy_blocks": (ctypes.c_int, [pkv_cache, pkv_cache, _c_vp, _c_i64, _c_vp]),
         "pkv_seq_block_table": (ctypes.c_int, [_c_vp, _c_i32, _c_vp, _c_i32, ctypes.POINTER(_c_i32)]),
         "pkv_seq_context_len": (_c_i64, [_c_vp, _c_i32]),
         "pkv_batch_tables": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_i32, _c_vp]),
@@ -303,6 +308,45 @@ def pkv_seq_append_slots(h, seqs):
     return out
 
 
+def pkv_seq_fork_tokens(h, parent: int, num_tokens: int) -> int:
+    s = ctypes.c_int32()
+    _check(lib.pkv_seq_fork_tokens(h, parent, num_tokens, ctypes.byref(s)), "pkv_seq_fork_tokens")
+    return s.value
+
+
+def pkv_seq_append_slot_cow(h, seq: int):
+    """(slot, copy_src, copy_dst); copy_src == -1 when no copy is needed."""
+    slot, src, dst = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.pkv_seq_append_slot_cow(h, seq, ctypes.byref(slot), ctypes.byref(src), ctypes.byref(dst)),
+           "pkv_seq_append_slot_cow")
+    return slot.value, src.value, dst.value
+
+
+def pkv_seq_append_slots_cow(h, seqs):
+    """(slots int64 [n], copies int32 [k][2]) for one new token of each sequence; all or nothing."""
+    import numpy as np
+
+    s = np.ascontiguousarray(seqs, dtype=np.int32)
+    slots = np.empty(len(s), dtype=np.int64)
+    copies = np.empty((max(1, len(s)), 2), dtype=np.int32)
+    nc = ctypes.c_int32()
+    _check(lib.pkv_seq_append_slots_cow(h, s.ctypes.data, len(s), slots.ctypes.data, copies.ctypes.data,
+                                        ctypes.byref(nc)), "pkv_seq_append_slots_cow")
+    return slots, copies[:nc.value].copy()
+
+
+def pkv_copy_blocks(k_cache, v_cache, pairs, stream=None) -> None:
+    """Copy whole blocks src -> dst (pairs: CUDA int32 [n][2]) in both pools."""
+    import torch
+
+    _require(pairs, "pairs")
+    if pairs.dtype != torch.int32:
+        raise TypeError("pairs must be int32")
+    n = pairs.numel() // 2
+    _check(lib.pkv_copy_blocks(cache_desc(k_cache), cache_desc(v_cache), pairs.data_ptr() if n else None, n,
+                               _stream_ptr(stream)), "pkv_copy_blocks")
+
+
 def pkv_seq_free(h, seq: int) -> None:
     _check(lib.pkv_seq_free(h, seq), "pkv_seq_free")
 
@@ -361,6 +405,9 @@ class BlockAllocator:
     append_slot = lambda self, s: pkv_seq_append_slot(self.handle, s)
     append_slots = lambda self, seqs: pkv_seq_append_slots(self.handle, seqs)
     seq_free = lambda self, s: pkv_seq_free(self.handle, s)
+    seq_fork_tokens = lambda self, p, n: pkv_seq_fork_tokens(self.handle, p, n)
+    append_slot_cow = lambda self, s: pkv_seq_append_slot_cow(self.handle, s)
+    append_slots_cow = lambda self, seqs: pkv_seq_append_slots_cow(self.handle, seqs)
     block_table = lambda self, s: pkv_seq_block_table(self.handle, s)
     context_len = lambda self, s: pkv_seq_context_len(self.handle, s)
     batch_tables = lambda self, seqs, cap: pkv_batch_tables(self.handle, seqs, cap)

@@ -11,9 +11,12 @@
 // Design: a LIFO free list of physical block ids, one reference count per
 // block (0 = free), and per-sequence logical->physical tables.  Sharing a
 // prefix is an incref of each shared block; a block returns to the free list
-// when its count reaches 0.  Only whole blocks are shared, and an append that
-// would land in a shared block is refused (PKV_ERR_SHARED_WRITE).  Every
-// operation either succeeds completely or leaves the state unchanged.
+// when its count reaches 0.  pkv_seq_fork shares whole blocks only, and a
+// plain append that would land in a shared block is refused
+// (PKV_ERR_SHARED_WRITE); pkv_seq_fork_tokens may share a partly filled last
+// block, and the copy-on-write appends give the writer a private copy (a
+// fresh block plus a device block copy the caller makes).  Every operation
+// either succeeds completely or leaves the state unchanged.
 #include <cstdint>
 #include <new>
 #include <vector>
@@ -207,6 +210,83 @@ pkv_status pkv_seq_append_slots(void *h, const int32_t *seqs, int32_t n, int64_t
         return PKV_ERR_OOM;
     for (int32_t i = 0; i < n; ++i)
         slots_out[i] = a->append_one(a->seqs[seqs[i]]);
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_fork_tokens(void *h, int32_t parent, int64_t num_tokens, int32_t *child_out) {
+    Allocator *a = as_alloc(h);
+    if (!a || !child_out || !a->valid_seq(parent) || num_tokens < 0)
+        return PKV_ERR_INVALID;
+    const Sequence &p = a->seqs[parent];
+    if (num_tokens > p.context_len)
+        return PKV_ERR_INVALID;
+    const int64_t nblk = (num_tokens + a->block_size - 1) / a->block_size;
+    std::vector<int32_t> shared(p.blocks.begin(), p.blocks.begin() + nblk);
+    int32_t id = a->new_seq_id();  // may grow seqs: do not hold references into it
+    Sequence &c = a->seqs[id];
+    c = Sequence();
+    c.live = true;
+    c.blocks = shared;
+    c.context_len = num_tokens;
+    for (int32_t b : shared)
+        a->refcount[b] += 1;
+    *child_out = id;
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_append_slot_cow(void *h, int32_t seq, int64_t *slot_out, int32_t *copy_src,
+                                   int32_t *copy_dst) {
+    Allocator *a = as_alloc(h);
+    if (!a || !slot_out || !copy_src || !copy_dst || !a->valid_seq(seq))
+        return PKV_ERR_INVALID;
+    Sequence &q = a->seqs[seq];
+    const bool shared = a->writes_shared(q);
+    if ((a->needs_block(q) || shared) && a->free_list.empty())
+        return PKV_ERR_OOM;
+    *copy_src = *copy_dst = -1;
+    if (shared) {
+        // copy-on-write: a private block replaces the shared one
+        const int64_t logical = q.context_len / a->block_size;
+        const int32_t old = q.blocks[logical];
+        const int32_t fresh = a->pop_block();
+        a->decref(old);
+        q.blocks[logical] = fresh;
+        *copy_src = old;
+        *copy_dst = fresh;
+    }
+    *slot_out = a->append_one(q);
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_append_slots_cow(void *h, const int32_t *seqs, int32_t n, int64_t *slots_out,
+                                    int32_t *copies_out, int32_t *n_copies_out) {
+    Allocator *a = as_alloc(h);
+    if (!a || n < 0 || !n_copies_out || (n > 0 && (!seqs || !slots_out || !copies_out)))
+        return PKV_ERR_INVALID;
+    std::vector<char> seen(a->seqs.size(), 0);
+    int64_t need = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t s = seqs[i];
+        if (!a->valid_seq(s) || seen[s])
+            return PKV_ERR_INVALID;
+        seen[s] = 1;
+        const Sequence &q = a->seqs[s];
+        if (a->needs_block(q) || a->writes_shared(q))
+            ++need;
+    }
+    if (need > (int64_t)a->free_list.size())
+        return PKV_ERR_OOM;
+    int32_t nc = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t src, dst;
+        pkv_seq_append_slot_cow(h, seqs[i], &slots_out[i], &src, &dst);  // cannot fail now
+        if (src >= 0) {
+            copies_out[2 * nc] = src;
+            copies_out[2 * nc + 1] = dst;
+            ++nc;
+        }
+    }
+    *n_copies_out = nc;
     return PKV_OK;
 }
 

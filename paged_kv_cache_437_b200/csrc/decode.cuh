@@ -1070,4 +1070,27 @@ __global__ void __launch_bounds__(256) append_kernel(const uint4 *__restrict__ k
     }
 }
 
+// ------------------------------------------------------------- block copy
+
+// Copy-on-write: whole blocks src -> dst in both pools, 16 bytes per thread.
+// A block is `chunks` 16-byte pieces, contiguous.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const int32_t *__restrict__ pairs, int64_t n,
+                                                          int64_t chunks, int64_t nb,
+                                                          uint4 *__restrict__ k_cache,
+                                                          uint4 *__restrict__ v_cache, unsigned *err) {
+    const int64_t total = n * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t p = i / chunks;
+        const int64_t c = i - p * chunks;
+        const int64_t src = __ldg(pairs + 2 * p), dst = __ldg(pairs + 2 * p + 1);
+        if (src < 0 || src >= nb || dst < 0 || dst >= nb) {
+            atomicOr(err, kErrSlot);
+            continue;
+        }
+        k_cache[dst * chunks + c] = k_cache[src * chunks + c];
+        v_cache[dst * chunks + c] = v_cache[src * chunks + c];
+    }
+}
+
 }  // namespace pkv

@@ -393,6 +393,31 @@ pkv_status pkv_append(const void *k_new, const void *v_new, const int64_t *slot_
     return cuda_ok(cudaGetLastError()) ? PKV_OK : PKV_ERR_CUDA;
 }
 
+pkv_status pkv_copy_blocks(pkv_cache k_cache, pkv_cache v_cache, const int32_t *pairs, int64_t num_pairs,
+                           pkv_stream stream) {
+    if (num_pairs < 0 || !cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
+        return PKV_ERR_INVALID;
+    if (num_pairs == 0)
+        return PKV_OK;
+    if (!pairs || (reinterpret_cast<uintptr_t>(pairs) & 7u))
+        return PKV_ERR_INVALID;
+    const int64_t block_bytes = k_cache.num_kv_heads * k_cache.block_size * k_cache.head_dim * 2;
+    if (block_bytes % 16)
+        return PKV_ERR_INVALID;
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+    const int64_t chunks = block_bytes / 16;
+    const int64_t total = num_pairs * chunks;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 32)
+        blocks = 148 * 32;
+    copy_blocks_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+        pairs, num_pairs, chunks, k_cache.num_blocks, static_cast<uint4 *>(k_cache.data),
+        static_cast<uint4 *>(v_cache.data), err);
+    return cuda_ok(cudaGetLastError()) ? PKV_OK : PKV_ERR_CUDA;
+}
+
 size_t pkv_decode_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
                                   int64_t head_dim, int64_t max_context_len,
                                   int32_t partition_tokens) {

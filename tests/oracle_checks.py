@@ -317,6 +317,18 @@ def check_split_merge(lib):
             assert np.max(np.abs(merged - full[0, h])) < 1e-12, (part, h)
 
 
+def check_copy_blocks(lib):
+    """Block copies against numpy fancy indexing, applied pair by pair."""
+    rng = np.random.default_rng(15)
+    pool = rng.integers(0, 65535, size=(7, 2, 4, 8), dtype=np.uint16)
+    exp = pool.copy()
+    pairs = np.array([[0, 3], [3, 5], [6, 0]], dtype=np.int32)
+    oracle.copy_blocks(pool, pairs, lib=lib)
+    for src, dst in pairs:
+        exp[dst] = exp[src]
+    assert np.array_equal(pool, exp)
+
+
 ALL_CHECKS = [check_decoders, check_sizing_golden, check_textbook, check_closed_forms, check_gqa_map,
               check_slot_bruteforce, check_append, check_permutation_and_sharing,
-              check_poison_and_scaling, check_split_merge]
+              check_poison_and_scaling, check_split_merge, check_copy_blocks]

@@ -185,3 +185,68 @@ def test_shuffled_free_list_via_public_api():
         a.decref(int(got[b]))
     again = [a.alloc() for _ in range(20)]
     assert again == [int(got[b]) for b in perm]
+
+
+def test_fork_tokens_and_copy_on_write():
+    a = pkv.BlockAllocator(8, 16)
+    p = a.seq_create()
+    for _ in range(20):                    # b0 full, b1 holds 4 tokens
+        a.append_slot(p)
+    b0, b1 = (int(x) for x in a.block_table(p))
+    c = a.seq_fork_tokens(p, 20)
+    assert list(a.block_table(c)) == [b0, b1] and a.context_len(c) == 20
+    assert a.refcount(b0) == 2 and a.refcount(b1) == 2
+    with pytest.raises(pkv.PkvError) as e:
+        a.append_slot(c)                   # plain append refuses the shared block
+    assert e.value.status == pkv.PKV_ERR_SHARED_WRITE
+    slot, src, dst = a.append_slot_cow(c)
+    assert src == b1 and dst not in (b0, b1)
+    assert list(a.block_table(c)) == [b0, dst] and slot == dst * 16 + 4
+    assert a.refcount(b1) == 1 and a.refcount(dst) == 1 and a.refcount(b0) == 2
+    slot_p, src_p, dst_p = a.append_slot_cow(p)   # parent's b1 is private again
+    assert (src_p, dst_p) == (-1, -1) and slot_p == b1 * 16 + 4
+    slot_c2, src2, _ = a.append_slot_cow(c)
+    assert src2 == -1 and slot_c2 == dst * 16 + 5
+    a.seq_free(p)
+    assert a.refcount(b0) == 1 and a.refcount(b1) == 0
+    a.seq_free(c)
+    assert a.num_free() == 8
+
+
+def test_copy_on_write_oom_changes_nothing():
+    a = pkv.BlockAllocator(2, 16)
+    p = a.seq_create()
+    for _ in range(5):
+        a.append_slot(p)
+    c = a.seq_fork_tokens(p, 5)
+    a.alloc()                              # the last free block
+    with pytest.raises(pkv.PkvError) as e:
+        a.append_slot_cow(c)
+    assert e.value.status == pkv.PKV_ERR_OOM
+    assert a.context_len(c) == 5 and a.refcount(int(a.block_table(c)[0])) == 2
+
+
+def test_batch_copy_on_write():
+    a = pkv.BlockAllocator(16, 16)
+    p = a.seq_create()
+    for _ in range(30):
+        a.append_slot(p)
+    kids = [a.seq_fork_tokens(p, n) for n in (30, 16, 7)]
+    slots, copies = a.append_slots_cow(kids)
+    # forks at 30 and 7 land in shared partial blocks; the fork at 16 opens a new block
+    assert len(copies) == 2
+    tables = [a.block_table(k) for k in kids]
+    assert slots[0] == tables[0][1] * 16 + 14 and slots[2] == tables[2][0] * 16 + 7
+    assert slots[1] == tables[1][1] * 16 + 0
+    srcs = sorted(int(x) for x in copies[:, 0])
+    assert srcs == sorted(int(x) for x in a.block_table(p)[:2][::-1])
+    full = pkv.BlockAllocator(3, 16)
+    q = full.seq_create()
+    for _ in range(20):
+        full.append_slot(q)
+    k1 = full.seq_fork_tokens(q, 20)
+    k2 = full.seq_fork_tokens(q, 20)
+    with pytest.raises(pkv.PkvError) as e:
+        full.append_slots_cow([k1, k2])    # needs two fresh blocks, one is free
+    assert e.value.status == pkv.PKV_ERR_OOM
+    assert full.context_len(k1) == 20 and full.context_len(k2) == 20

@@ -28,6 +28,8 @@ MUTATIONS = {
     "merge_weight_dropped": ("total += l[j] * w;", "total += l[j];"),
     "not_normalised": ("o[d] = o[d] / l;", "o[d] = o[d];"),
     "max_not_subtracted_sign": ("double w = exp(z[i] - m);", "double w = exp(m - z[i]);"),
+    "copy_blocks_swapped": ("memmove(cache + dst * block_elems, cache + src * block_elems,",
+                            "memmove(cache + src * block_elems, cache + dst * block_elems,"),
     "kv_sizing_factor": ("return 2 * seq_len * kv_heads * head_dim * dtype_bytes;",
                          "return seq_len * kv_heads * head_dim * dtype_bytes;"),
 }
