@@ -611,6 +611,104 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ main
 
+# ------------------------------------------------------------------ NEXT rows
+
+def run_row(args) -> dict:
+    """Measurements of the rows next to the hot path (one JSON line each)."""
+    import torch
+
+    import paged_kv_cache_437_b200 as pkv
+    import workloads
+
+    rng = np.random.default_rng(5)
+    if args.row == "sched":
+        alloc = pkv.BlockAllocator(65536, 16)
+        sched = pkv.Scheduler(alloc, max_batch_tokens=8192, max_seqs=256, chunk_tokens=512)
+        lens = np.clip(np.exp(rng.uniform(np.log(16), np.log(4096), 1024)), 16, 4096).astype(int)
+        for i, p in enumerate(lens):
+            sched.add(i, int(p), int(rng.integers(16, 256)))
+        t0 = time.perf_counter()
+        steps = tokens = 0
+        while (sched.num_waiting or sched.num_running) and steps < 2000:
+            b = sched.step()
+            steps += 1
+            tokens += len(b["slots"])
+        dt = time.perf_counter() - t0
+        return {"row": "scheduler", "metric": "host scheduler step time", "value": round(dt / steps * 1e6, 2),
+                "unit": "us/step", "higher_is_better": False, "steps": steps, "tokens": tokens,
+                "config": {"requests": 1024, "prompt": "log-uniform [16, 4096]", "max_new": "uniform [16, 256)",
+                           "max_batch_tokens": 8192, "max_seqs": 256, "chunk_tokens": 512, "pool_blocks": 65536}}
+
+    torch.cuda.set_device(0)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    if args.row == "cow":
+        nb, hkv, bs, d = 8192, 40, 16, 128          # 13B-shaped blocks: 160 KB of K + 160 KB of V
+        kc = torch.randn((nb, hkv, bs, d), dtype=torch.float16, device="cuda")
+        vc = torch.randn_like(kc)
+        n = 2048
+        perm = rng.permutation(nb)
+        pairs = torch.from_numpy(np.stack([perm[:n], perm[n:2 * n]], 1).astype(np.int32)).cuda()
+        for _ in range(args.warmup):
+            pkv.pkv_copy_blocks(kc, vc, pairs)
+        t0, t1 = ev(), ev()
+        t0.record()
+        for _ in range(args.steps):
+            pkv.pkv_copy_blocks(kc, vc, pairs)
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / args.steps
+        moved = n * 2 * (hkv * bs * d * 2) * 2     # read + write of K and V blocks
+        return {"row": "copy_on_write", "metric": "block copy HBM GB/s (read + write)",
+                "value": round(moved / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "ms_per_call": round(ms, 4),
+                "peak": load_peaks()["hbm_gbs"], "config": {"pairs": n, "block": [hkv, bs, d], "dtype": "f16"}}
+
+    if args.row == "prefill":
+        # 70B-shaped layer: 2 prompts of a 2048-token prefix + one 512-token
+        # chunk each, interleaved with 30 decode sequences of 4096 context
+        hq, hkv, d, bs = 64, 8, 128, 16
+        chunks = [(2048 + 512, 512)] * 2 + [(4096, 1)] * 30
+        ctx = np.array([c for c, _ in chunks], np.int32)
+        nq = np.array([n for _, n in chunks], np.int32)
+        qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+        t = int(qs[-1])
+        nblk = -(-ctx // bs)
+        mb = int(nblk.max())
+        nb = int(nblk.sum()) + 8
+        perm = rng.permutation(nb).astype(np.int32)
+        tables = np.full((len(chunks), mb), -1, np.int32)
+        cur = 0
+        for i, k in enumerate(nblk):
+            tables[i, :k] = perm[cur:cur + k]
+            cur += k
+        kc = torch.randn((nb, hkv, bs, d), dtype=torch.bfloat16, device="cuda")
+        vc = torch.randn_like(kc)
+        q = torch.randn((t, hq, d), dtype=torch.bfloat16, device="cuda")
+        out = torch.empty_like(q)
+        ws = torch.empty(pkv.pkv_prefill_workspace_bytes(t, hq, hkv, d, mb * bs), dtype=torch.uint8, device="cuda")
+        td, qsd, cd = (torch.from_numpy(x).cuda() for x in (tables, qs, ctx))
+        for _ in range(args.warmup):
+            pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
+        t0, t1 = ev(), ev()
+        t0.record()
+        for _ in range(args.steps):
+            pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / args.steps
+        # work: each query token attends to its causal window
+        windows = np.concatenate([np.arange(c - n + 1, c + 1) for c, n in chunks]).astype(np.int64)
+        flops = int(windows.sum()) * hq * d * 2 * 2
+        unique = int((ctx.astype(np.int64)).sum()) * hkv * d * 2 * 2
+        return {"row": "chunked_prefill", "metric": "chunked prefill + decode step: query tokens/s",
+                "value": round(t / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+                "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "unique_kv_gbs": round(unique / (ms * 1e-3) / 1e9, 1),
+                "bf16_peak_tflops": json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"]
+                if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None,
+                "config": {"shape": "70B GQA 64/8, D128, bs16, bf16", "prefill": "2 x (2048 prefix + 512 chunk)",
+                           "decode": "30 x 4096", "query_tokens": t}}
+    raise SystemExit(f"unknown row {args.row}")
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -621,6 +719,8 @@ def parse_args(argv=None):
                     help="partition tokens: 0 auto (default), -1 none, P > 0 fixed P-token partitions")
     ap.add_argument("--flush-l2", action="store_true")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--row", default=None, choices=["cow", "prefill", "sched", "fp8"],
+                    help="measure a row next to the hot path instead (one JSON line tagged 'row')")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass (profiling runs)")
@@ -641,6 +741,10 @@ def parse_args(argv=None):
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
+    if args.row:
+        if rank == 0:
+            print(json.dumps(run_row(args)), flush=True)
+        return 0
     if args.impl == "reference":
         if rank != 0:
             return 0

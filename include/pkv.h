@@ -183,6 +183,37 @@ pkv_status pkv_append_decode_attention(const void *k_new, const void *v_new,
                                        int32_t partition_tokens, pkv_stream stream);
 
 /* --------------------------------------------------------------------------
+ * pkv_prefill_attention -- chunked prefill over the paged cache.
+ * [KVB] "Chunked prefill": a long prompt is split into fixed-size chunks
+ * (e.g. 512 tokens) that are interleaved with other requests' decode steps.
+ *
+ *   q, out         device [T][Hq][D], the chunk tokens of all sequences in
+ *                  sequence order, T = num_tokens = query_start[B]
+ *   query_start    device int32 [B + 1], query_start[0] = 0: sequence s owns
+ *                  tokens query_start[s] .. query_start[s+1] - 1 (n_s >= 1)
+ *   context_lens   device int32 [B]: length of sequence s AFTER its chunk's
+ *                  K/V were appended (pkv_append with the chunk's slots), so
+ *                  the chunk holds positions ctx_s - n_s .. ctx_s - 1
+ *   block_tables   device int32 [B][MB], one row per sequence
+ *   workspace      required, >= pkv_prefill_workspace_bytes(...)
+ *
+ * Query i of sequence s attends causally to positions 0 .. ctx_s - n_s + i.
+ * A decode sequence is a chunk of one, so prefill chunks and decode tokens
+ * go in one call.  Each query token runs as its own decode over its causal
+ * prefix (sharing the sequence's table row), on the decode kernel; the
+ * chunk's tokens re-read the shared prefix, mostly from L2.  Inconsistent
+ * lengths (n_s < 1, ctx_s < n_s) are flagged on the device and give zero
+ * rows.  Same limits as pkv_decode_attention; T < 2^24.
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_seqs, int64_t num_q_heads,
+                                 pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+                                 int64_t max_blocks_per_seq, const int32_t *query_start,
+                                 const int32_t *context_lens, float scale, void *out, void *workspace,
+                                 size_t workspace_bytes, pkv_stream stream);
+size_t pkv_prefill_workspace_bytes(int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
+                                   int64_t head_dim, int64_t max_context_len);
+
+/* --------------------------------------------------------------------------
  * pkv_decode_attention_static_scratch -- pkv_decode_attention for callers
  * that cannot allocate device memory.  (No counterpart on the pages: this is
  * an interface convenience, not part of the method.)
@@ -314,6 +345,57 @@ pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns);
 /* Text of the last CUDA runtime error a call of this thread reported as
  * PKV_ERR_CUDA ("no error" if none); static storage. */
 const char *pkv_last_cuda_error(void);
+
+/* --------------------------------------------------------------------------
+ * Iteration-level scheduler (host only) over one allocator.
+ * [KVB] "Continuous batching (Orca)": each token step is batched across all
+ * in-flight requests; finished requests leave and new ones join at any step.
+ * [KVB] "Chunked prefill": prompts are fed in fixed-size chunks interleaved
+ * with decode steps.  [KVB] "The KV cache": running out of KV memory stalls
+ * new requests or forces preemption of in-flight ones.
+ *
+ * Each pkv_sched_step plans one step: one decode token for every request
+ * past its prompt (oldest first), then the next prefill chunk (<=
+ * chunk_tokens) of requests still in their prompt, then new requests first
+ * come first served -- within max_batch_tokens tokens and max_seqs
+ * sequences.  When a request needs a block and none is free, the most
+ * recently admitted other request is preempted by recompute (its blocks
+ * return to the pool; it rejoins the front of the queue and re-prefills its
+ * prompt and generated tokens).  The step's slots come from the allocator,
+ * so pkv_batch_tables(seq_ids) gives the matching block tables; run
+ * pkv_append with the slots, then pkv_prefill_attention with query_lens as
+ * the chunk lengths (a decode token is a chunk of one).  The step that
+ * completes a request's context produces its next token; a request that
+ * reached max_new_tokens is reported in finished_ids by the NEXT call, which
+ * also frees its blocks (this step's kernels still read them).
+ * ------------------------------------------------------------------------ */
+typedef struct pkv_sched_config {
+    int32_t max_batch_tokens;  /* tokens per step (decode tokens + prefill chunks) */
+    int32_t max_seqs;          /* sequences per step and requests running at once */
+    int32_t chunk_tokens;      /* prefill chunk size, e.g. 512 */
+    int32_t block_size;        /* the allocator's block size */
+} pkv_sched_config;
+
+/* Caller-owned output arrays of one step; capacities: max_seqs entries for
+ * the per-sequence arrays, max_batch_tokens for slots. */
+typedef struct pkv_sched_batch {
+    int32_t num_seqs, num_tokens, num_preempted, num_finished;
+    int64_t *request_ids;   /* [max_seqs] */
+    int32_t *seq_ids;       /* [max_seqs] allocator sequence ids */
+    int32_t *query_lens;    /* [max_seqs] tokens of the sequence in this step */
+    int32_t *context_lens;  /* [max_seqs] sequence length after this step */
+    int64_t *slots;         /* [max_batch_tokens] new tokens' slots, sequence order */
+    int64_t *finished_ids;  /* [max_seqs] */
+    int64_t *preempted_ids; /* [max_seqs] */
+} pkv_sched_batch;
+
+pkv_status pkv_sched_create(void *alloc, const pkv_sched_config *cfg, void **sched);
+void pkv_sched_destroy(void *sched);
+/* Queue a request: prompt_len prompt tokens, then max_new_tokens outputs. */
+pkv_status pkv_sched_add(void *sched, int64_t request_id, int32_t prompt_len, int32_t max_new_tokens);
+pkv_status pkv_sched_step(void *sched, pkv_sched_batch *out);
+int32_t pkv_sched_num_waiting(void *sched);
+int32_t pkv_sched_num_running(void *sched);
 
 /* Human-readable name of a status code (static storage). */
 const char *pkv_status_string(pkv_status s);

@@ -58,6 +58,9 @@ def _bind(lib):
         vp, i64, vp]
     lib.oracle_lse_merge.restype = ctypes.c_int
     lib.oracle_lse_merge.argtypes = [i64, vp, vp, vp, i64, vp]
+    lib.oracle_prefill_attention.restype = ctypes.c_int
+    lib.oracle_prefill_attention.argtypes = [ctypes.c_int, vp, i64, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64,
+                                             vp, vp, dbl, vp]
     lib.oracle_copy_blocks.restype = ctypes.c_int
     lib.oracle_copy_blocks.argtypes = [vp, i64, i64, vp, i64]
     lib.oracle_mark_slots.restype = ctypes.c_int
@@ -206,6 +209,25 @@ def slot_mask(block_tables, lens, block_size: int, num_blocks: int, lib=None) ->
     if rc != 0:
         raise ValueError("oracle_mark_slots: table entry out of range")
     return mask.astype(bool)
+
+
+def prefill_attention(q, k_cache, v_cache, block_tables, query_start, context_lens, scale, dtype,
+                      lib=None) -> np.ndarray:
+    """Causal chunked-prefill attention, fp64 [T][Hq][D] (see the C source)."""
+    lib = lib or load()
+    q16 = _u16(q)
+    t, hq, d = q16.shape
+    k16, v16 = _u16(k_cache), _u16(v_cache)
+    nb, hkv, bs, _ = k16.shape
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    rc = lib.oracle_prefill_attention(dtype, _p(q16), t, len(cl), hq, _p(k16), _p(v16), nb, bs, hkv, d, _p(bt),
+                                      bt.shape[1], _p(qs), _p(cl), float(scale), _p(out))
+    if rc != 0:
+        raise ValueError("oracle_prefill_attention: inconsistent lengths or table entry out of range")
+    return out
 
 
 def copy_blocks(cache: np.ndarray, pairs, lib=None) -> None:

@@ -367,3 +367,59 @@ int oracle_copy_blocks(uint16_t *cache, int64_t num_blocks, int64_t block_elems,
     }
     return 0;
 }
+
+/*
+ * Chunked prefill attention ("LLM Inference: KV Cache, Batching &
+ * Scheduling", cariara.com, section "Chunked prefill": a prompt is split
+ * into fixed-size chunks interleaved with decode steps).  Sequence s has
+ * n_s = query_start[s+1] - query_start[s] new query tokens whose K/V are
+ * already in the cache at positions ctx_s - n_s .. ctx_s - 1; query i of the
+ * chunk attends to positions 0 .. ctx_s - n_s + i (causal).  A decode
+ * sequence is a chunk of one.  q and out are [T][Hq][D] with
+ * T = query_start[B]; out is fp64.  Returns -1 on inconsistent lengths.
+ */
+int oracle_prefill_attention(int dtype, const uint16_t *q, int64_t num_tokens,
+                             int64_t num_seqs, int64_t num_q_heads,
+                             const uint16_t *k_cache, const uint16_t *v_cache,
+                             int64_t num_blocks, int64_t block_size,
+                             int64_t num_kv_heads, int64_t head_dim,
+                             const int32_t *block_tables, int64_t max_blocks_per_seq,
+                             const int32_t *query_start, const int32_t *context_lens,
+                             double scale, double *out)
+{
+    if (query_start[0] != 0 || query_start[num_seqs] != num_tokens)
+        return -1;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t n = query_start[s + 1] - query_start[s];
+        int64_t ctx = context_lens[s];
+        if (n < 0 || ctx < n) {
+            err |= 1;
+            continue;
+        }
+        for (int64_t i = 0; i < n; ++i) {
+            int64_t tok = query_start[s] + i;
+            int64_t window = ctx - n + i + 1;     /* positions 0 .. ctx - n + i */
+            for (int64_t h = 0; h < num_q_heads; ++h) {
+                double m, l;
+                double *o = out + (tok * num_q_heads + h) * head_dim;
+                /* the query row of token tok, head h sits at q[tok][h]: call
+                 * the range routine with the token's row as "sequence" */
+                if (oracle_attention_range(dtype, q + tok * num_q_heads * head_dim, num_q_heads,
+                                           k_cache, v_cache, num_blocks, block_size,
+                                           num_kv_heads, head_dim,
+                                           block_tables + s * max_blocks_per_seq,
+                                           max_blocks_per_seq, scale, 0, h, 0, window,
+                                           &m, &l, o)) {
+                    err |= 1;
+                    continue;
+                }
+                if (l > 0.0)
+                    for (int64_t d = 0; d < head_dim; ++d)
+                        o[d] /= l;
+            }
+        }
+    }
+    return err ? -1 : 0;
+}

@@ -41,6 +41,18 @@ class pkv_cache(ctypes.Structure):
                 ("head_dim", ctypes.c_int64)]
 
 
+class pkv_sched_config(ctypes.Structure):
+    _fields_ = [("max_batch_tokens", ctypes.c_int32), ("max_seqs", ctypes.c_int32),
+                ("chunk_tokens", ctypes.c_int32), ("block_size", ctypes.c_int32)]
+
+
+class pkv_sched_batch(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_tokens", ctypes.c_int32), ("num_preempted", ctypes.c_int32),
+                ("num_finished", ctypes.c_int32), ("request_ids", ctypes.c_void_p), ("seq_ids", ctypes.c_void_p),
+                ("query_lens", ctypes.c_void_p), ("context_lens", ctypes.c_void_p), ("slots", ctypes.c_void_p),
+                ("finished_ids", ctypes.c_void_p), ("preempted_ids", ctypes.c_void_p)]
+
+
 class PkvError(RuntimeError):
     def __init__(self, status: int, what: str):
         detail = f" [{lib.pkv_last_cuda_error().decode()}]" if status == PKV_ERR_CUDA else ""
@@ -77,6 +89,16 @@ def _load():
                                                    ctypes.POINTER(_c_i32)]),
         "pkv_seq_append_slots_cow": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp, ctypes.POINTER(_c_i32)]),
         "pkv_copy_blocks": (ctypes.c_int, [pkv_cache, pkv_cache, _c_vp, _c_i64, _c_vp]),
+        "pkv_sched_create": (ctypes.c_int, [_c_vp, ctypes.POINTER(pkv_sched_config), ctypes.POINTER(_c_vp)]),
+        "pkv_sched_destroy": (None, [_c_vp]),
+        "pkv_sched_add": (ctypes.c_int, [_c_vp, _c_i64, _c_i32, _c_i32]),
+        "pkv_sched_step": (ctypes.c_int, [_c_vp, ctypes.POINTER(pkv_sched_batch)]),
+        "pkv_sched_num_waiting": (_c_i32, [_c_vp]),
+        "pkv_sched_num_running": (_c_i32, [_c_vp]),
+        "pkv_prefill_attention": (ctypes.c_int, [_c_vp, _c_i64, _c_i64, _c_i64, pkv_cache, pkv_cache, _c_vp,
+                                                 _c_i64, _c_vp, _c_vp, ctypes.c_float, _c_vp, _c_vp, _c_sz,
+                                                 _c_vp]),
+        "pkv_prefill_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64]),
         "pkv_seq_block_table": (ctypes.c_int, [_c_vp, _c_i32, _c_vp, _c_i32, ctypes.POINTER(_c_i32)]),
         "pkv_seq_context_len": (_c_i64, [_c_vp, _c_i32]),
         "pkv_batch_tables": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_i32, _c_vp]),
@@ -239,6 +261,31 @@ def pkv_append_decode_attention(k_new, v_new, slot_mapping, q, k_cache, v_cache,
                                          float(scale), out.data_ptr(), ws_ptr or None, ws_bytes,
                                          int(partition_tokens), _stream_ptr(stream))
     _check(st, "pkv_append_decode_attention")
+
+
+def pkv_prefill_workspace_bytes(num_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                max_context_len: int) -> int:
+    return int(lib.pkv_prefill_workspace_bytes(num_tokens, num_q_heads, num_kv_heads, head_dim, max_context_len))
+
+
+def pkv_prefill_attention(q, k_cache, v_cache, block_tables, query_start, context_lens, scale: float, out,
+                          workspace, stream=None) -> None:
+    """Causal chunked-prefill attention: q/out [T][Hq][D], query_start [B+1], context_lens [B]."""
+    import torch
+
+    for t, n in ((q, "q"), (out, "out"), (block_tables, "block_tables"), (query_start, "query_start"),
+                 (context_lens, "context_lens"), (workspace, "workspace")):
+        _require(t, n)
+    if query_start.dtype != torch.int32 or context_lens.dtype != torch.int32 or block_tables.dtype != torch.int32:
+        raise TypeError("query_start, context_lens and block_tables must be int32")
+    b = context_lens.numel()
+    if query_start.numel() != b + 1 or block_tables.shape[0] != b or out.shape != q.shape or q.dim() != 3:
+        raise ValueError("shapes: q/out [T][Hq][D], query_start [B+1], context_lens [B], block_tables [B][MB]")
+    st = lib.pkv_prefill_attention(q.data_ptr(), q.shape[0], b, q.shape[1], cache_desc(k_cache), cache_desc(v_cache),
+                                   block_tables.data_ptr(), block_tables.shape[1], query_start.data_ptr(),
+                                   context_lens.data_ptr(), float(scale), out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(st, "pkv_prefill_attention")
 
 
 def pkv_get_last_error() -> int:
@@ -411,3 +458,53 @@ class BlockAllocator:
     block_table = lambda self, s: pkv_seq_block_table(self.handle, s)
     context_len = lambda self, s: pkv_seq_context_len(self.handle, s)
     batch_tables = lambda self, seqs, cap: pkv_batch_tables(self.handle, seqs, cap)
+
+
+class Scheduler:
+    """Iteration-level scheduler over a BlockAllocator (host only)."""
+
+    def __init__(self, alloc: "BlockAllocator", max_batch_tokens: int, max_seqs: int, chunk_tokens: int = 512):
+        import numpy as np
+
+        self.alloc = alloc
+        self.cfg = pkv_sched_config(max_batch_tokens, max_seqs, chunk_tokens, alloc.block_size)
+        h = ctypes.c_void_p()
+        _check(lib.pkv_sched_create(alloc.handle, ctypes.byref(self.cfg), ctypes.byref(h)), "pkv_sched_create")
+        self.handle = h
+        self._arr = dict(request_ids=np.zeros(max_seqs, np.int64), seq_ids=np.zeros(max_seqs, np.int32),
+                         query_lens=np.zeros(max_seqs, np.int32), context_lens=np.zeros(max_seqs, np.int32),
+                         slots=np.zeros(max_batch_tokens, np.int64), finished_ids=np.zeros(max_seqs, np.int64),
+                         preempted_ids=np.zeros(max_seqs, np.int64))
+        self._batch = pkv_sched_batch(0, 0, 0, 0, *(self._arr[k].ctypes.data for k in (
+            "request_ids", "seq_ids", "query_lens", "context_lens", "slots", "finished_ids", "preempted_ids")))
+
+    def add(self, request_id: int, prompt_len: int, max_new_tokens: int) -> None:
+        _check(lib.pkv_sched_add(self.handle, request_id, prompt_len, max_new_tokens), "pkv_sched_add")
+
+    def step(self) -> dict:
+        _check(lib.pkv_sched_step(self.handle, ctypes.byref(self._batch)), "pkv_sched_step")
+        b, a = self._batch, self._arr
+        return dict(request_ids=a["request_ids"][:b.num_seqs].copy(), seq_ids=a["seq_ids"][:b.num_seqs].copy(),
+                    query_lens=a["query_lens"][:b.num_seqs].copy(),
+                    context_lens=a["context_lens"][:b.num_seqs].copy(), slots=a["slots"][:b.num_tokens].copy(),
+                    finished=a["finished_ids"][:b.num_finished].copy(),
+                    preempted=a["preempted_ids"][:b.num_preempted].copy())
+
+    @property
+    def num_waiting(self) -> int:
+        return int(lib.pkv_sched_num_waiting(self.handle))
+
+    @property
+    def num_running(self) -> int:
+        return int(lib.pkv_sched_num_running(self.handle))
+
+    def close(self):
+        if self.handle:
+            lib.pkv_sched_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -83,6 +83,9 @@ struct DecodeArgs {
     const int64_t *slots;          // [B], < 0: no append for that sequence
     uint16_t *k_cache, *v_cache;   // the pools, for the generic-store append
     int64_t pool_slots;            // NB * bs
+    // chunked prefill: "sequence" s reads block-table row table_rows[s]
+    // (several query tokens of one sequence share its row); null = row s
+    const int32_t *table_rows;
 };
 
 struct SmemLayout {
@@ -134,6 +137,7 @@ __device__ __forceinline__ int upper_bound_i(const int *a, int n, long long x) {
 
 struct Seg {
     int seq, pair, t0, t1, ctx, dest;  // dest < 0: final output, else partial index
+    int trow;                          // block-table row of the sequence
 };
 
 struct Walker {
@@ -167,8 +171,19 @@ __device__ __forceinline__ void walker_init(Walker &w, const DecodeArgs &a, cons
     }
 }
 
+__device__ __forceinline__ bool walker_next_raw(Walker &w, Seg &sg, const DecodeArgs &a,
+                                                const int *prefix, const int *ctxs, int gw);
+
 __device__ __forceinline__ bool walker_next(Walker &w, Seg &sg, const DecodeArgs &a,
                                             const int *prefix, const int *ctxs, int gw) {
+    const bool has = walker_next_raw(w, sg, a, prefix, ctxs, gw);
+    if (has)
+        sg.trow = a.table_rows ? __ldg(a.table_rows + sg.seq) : sg.seq;
+    return has;
+}
+
+__device__ __forceinline__ bool walker_next_raw(Walker &w, Seg &sg, const DecodeArgs &a,
+                                                const int *prefix, const int *ctxs, int gw) {
     if (a.mode == kModeDirect) {
         if (w.u >= (long long)a.B * a.npairs)
             return false;
@@ -388,7 +403,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const int nblk = ceil_div_i(ns.ctx, a.bs);
             nx_seq = ns.seq;
             nx_base = lb;
-            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.seq * a.mb + lb + lane) : 0;
+            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.trow * a.mb + lb + lane) : 0;
         }
     };
     // set when the producer enters a unit; the prefetch for the unit after it
@@ -407,7 +422,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 nx_seq = -1;
             } else {
                 const int nblk = ceil_div_i(ps.ctx, a.bs);
-                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.seq * a.mb + lb + lane) : 0;
+                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.trow * a.mb + lb + lane) : 0;
             }
         }
         if (want_prefetch) {
@@ -1090,6 +1105,39 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const int32_t *__restr
         }
         k_cache[dst * chunks + c] = k_cache[src * chunks + c];
         v_cache[dst * chunks + c] = v_cache[src * chunks + c];
+    }
+}
+
+// ------------------------------------------------------------- chunked prefill
+
+// Query token j of sequence s (chunk of n tokens, context ctx after the
+// chunk's append) attends to positions 0 .. ctx - n + i: a decode of length
+// ctx - n + i + 1 over row s of the block table.
+__global__ void __launch_bounds__(256) prefill_expand_kernel(const int32_t *__restrict__ query_start,
+                                                             const int32_t *__restrict__ context_lens,
+                                                             int B, int T, int64_t cap,
+                                                             int32_t *__restrict__ lens,
+                                                             int32_t *__restrict__ rows, unsigned *err) {
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < T; j += gridDim.x * blockDim.x) {
+        int lo = 0, hi = B + 1;  // first index with query_start > j
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(query_start + mid) <= j)
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        const int s = max(0, min(B - 1, lo - 1));
+        const int q0 = __ldg(query_start + s);
+        const int n = __ldg(query_start + s + 1) - q0;
+        const int c = __ldg(context_lens + s);
+        int len = c - n + (j - q0) + 1;
+        if (n <= 0 || c < n || c > cap || j < q0 || j >= q0 + n) {
+            atomicOr(err, kErrContext);
+            len = 0;
+        }
+        lens[j] = len;
+        rows[j] = s;
     }
 }
 

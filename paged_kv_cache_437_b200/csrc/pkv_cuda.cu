@@ -448,7 +448,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
                        pkv_cache v_cache, const int32_t *block_tables, int64_t max_blocks_per_seq,
                        const int32_t *context_lens, float scale, void *out, void *workspace,
                        size_t workspace_bytes, int32_t partition_tokens, pkv_stream stream,
-                       const FusedAppend *fa) {
+                       const FusedAppend *fa, const int32_t *table_rows = nullptr) {
     if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0)
         return PKV_ERR_INVALID;
     if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
@@ -538,6 +538,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.k_cache = static_cast<uint16_t *>(k_cache.data);
     a.v_cache = static_cast<uint16_t *>(v_cache.data);
     a.pool_slots = k_cache.num_blocks * bs;
+    a.table_rows = table_rows;
 
     DecodeKernel k = pick_decode((int)D, bf16, p.nt);
     if (!cuda_ok(launch_dependent(k, dim3(p.ctas), dim3(p.warps * 32), p.smem, (cudaStream_t)stream, tmK,
@@ -619,6 +620,49 @@ pkv_status pkv_append_decode_attention(const void *k_new, const void *v_new,
 }
 
 const char *pkv_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
+size_t pkv_prefill_workspace_bytes(int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
+                                   int64_t head_dim, int64_t max_context_len) {
+    if (num_tokens < 0)
+        return 0;
+    const size_t dec = pkv_decode_workspace_bytes(num_tokens, num_q_heads, num_kv_heads, head_dim,
+                                                  max_context_len, PKV_PARTITION_AUTO);
+    if (dec == 0 && num_tokens > 0)
+        return 0;
+    return align256((size_t)num_tokens * 8) + dec;
+}
+
+pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_seqs, int64_t num_q_heads,
+                                 pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+                                 int64_t max_blocks_per_seq, const int32_t *query_start,
+                                 const int32_t *context_lens, float scale, void *out, void *workspace,
+                                 size_t workspace_bytes, pkv_stream stream) {
+    if (num_tokens < 0 || num_seqs < 0 || num_tokens >= (int64_t(1) << 24))
+        return PKV_ERR_INVALID;
+    if (num_tokens == 0)
+        return PKV_OK;
+    if (num_seqs == 0 || !query_start || !context_lens || !workspace || !aligned16(workspace) ||
+        !cache_ok(k_cache) || (reinterpret_cast<uintptr_t>(query_start) & 3u))
+        return PKV_ERR_INVALID;
+    const size_t head = align256((size_t)num_tokens * 8);
+    if (workspace_bytes < head)
+        return PKV_ERR_INVALID;
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+    int32_t *lens = static_cast<int32_t *>(workspace);
+    int32_t *rows = lens + num_tokens;
+    const int64_t blocks = std::min<int64_t>((num_tokens + 255) / 256, 148 * 8);
+    prefill_expand_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+        query_start, context_lens, (int)num_seqs, (int)num_tokens, max_blocks_per_seq * k_cache.block_size,
+        lens, rows, err);
+    if (!cuda_ok(cudaGetLastError()))
+        return PKV_ERR_CUDA;
+    char *rest = static_cast<char *>(workspace) + head;
+    return decode_impl(q, num_tokens, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq, lens,
+                       scale, out, workspace_bytes > head ? rest : nullptr, workspace_bytes - head,
+                       PKV_PARTITION_AUTO, stream, nullptr, rows);
+}
 
 pkv_status pkv_get_last_error(void) {
     if (!cuda_ok(cudaDeviceSynchronize()))

@@ -329,6 +329,34 @@ def check_copy_blocks(lib):
     assert np.array_equal(pool, exp)
 
 
+def check_prefill(lib):
+    """Chunked prefill: scipy softmax over each query's causal window on the
+    unpaged caches, and a chunk of one equals the decode oracle."""
+    rng = np.random.default_rng(16)
+    b, hq, hkv, d, bs, n = 3, 4, 2, 8, 4, 16
+    q_all, k, v = _rand_case(rng, 6, hq, hkv, d, n, oracle.BF16)
+    k, v = k[:b], v[:b]
+    ctx = np.array([16, 9, 5], dtype=np.int32)
+    nq = [5, 1, 0]                                    # chunk lengths
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = q_all[:qs[-1]]
+    kp, vp = contiguous_to_pool(k, bs), contiguous_to_pool(v, bs)
+    tables = np.arange(b * n // bs, dtype=np.int32).reshape(b, n // bs)
+    got = oracle.prefill_attention(q, kp, vp, tables, qs, ctx, 0.4, oracle.BF16, lib=lib)
+    kd, vd, qd = bits_to_f64(k, oracle.BF16), bits_to_f64(v, oracle.BF16), bits_to_f64(q, oracle.BF16)
+    grp = hq // hkv
+    for s in range(b):
+        for i in range(nq[s]):
+            tok = qs[s] + i
+            win = ctx[s] - nq[s] + i + 1
+            for h in range(hq):
+                p = scipy.special.softmax(0.4 * (kd[s, h // grp, :win] @ qd[tok, h]))
+                assert np.max(np.abs(got[tok, h] - p @ vd[s, h // grp, :win])) < 1e-12
+    # the one-token chunk of sequence 1 is a decode over its whole context
+    dec = oracle.attention(q[qs[1]:qs[1] + 1], kp, vp, tables[1:2], ctx[1:2], 0.4, oracle.BF16, lib=lib)
+    assert np.array_equal(dec[0], got[qs[1]])
+
+
 ALL_CHECKS = [check_decoders, check_sizing_golden, check_textbook, check_closed_forms, check_gqa_map,
               check_slot_bruteforce, check_append, check_permutation_and_sharing,
-              check_poison_and_scaling, check_split_merge, check_copy_blocks]
+              check_poison_and_scaling, check_split_merge, check_copy_blocks, check_prefill]

@@ -30,6 +30,7 @@ MUTATIONS = {
     "max_not_subtracted_sign": ("double w = exp(z[i] - m);", "double w = exp(m - z[i]);"),
     "copy_blocks_swapped": ("memmove(cache + dst * block_elems, cache + src * block_elems,",
                             "memmove(cache + src * block_elems, cache + dst * block_elems,"),
+    "prefill_window_off_by_one": ("int64_t window = ctx - n + i + 1;", "int64_t window = ctx - n + i;"),
     "kv_sizing_factor": ("return 2 * seq_len * kv_heads * head_dim * dtype_bytes;",
                          "return seq_len * kv_heads * head_dim * dtype_bytes;"),
 }
