@@ -706,6 +706,67 @@ def run_row(args) -> dict:
                 if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None,
                 "config": {"shape": "70B GQA 64/8, D128, bs16, bf16", "prefill": "2 x (2048 prefix + 512 chunk)",
                            "decode": "30 x 4096", "query_tokens": t}}
+
+    if args.row == "fp8":
+        # the workload's decode over E4M3 pools (1 byte per element + one fp32
+        # scale per row) beside the same decode over its 16-bit pools; K
+        # launches back to back between two events, like the dominant-kernel
+        # loop of the main step (both working sets are larger than L2)
+        w = make_workload(args)
+        sp = w.spec
+        dt = torch.float16 if sp.dtype == workloads.F16 else torch.bfloat16
+        dev16 = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).cuda()
+        shape = w.k_cache.shape
+        gen = torch.Generator(device="cuda").manual_seed(11)
+
+        def codes():  # any finite E4M3 code: magnitude bits 0x00..0x7e, random sign
+            mag = torch.randint(0, 0x7f, shape, generator=gen, device="cuda", dtype=torch.int16)
+            sign = torch.randint(0, 2, shape, generator=gen, device="cuda", dtype=torch.int16) << 7
+            return (mag | sign).to(torch.uint8)
+
+        k8, v8 = codes(), codes()
+        ks = torch.rand(shape[:3], generator=gen, device="cuda") * 0.01 + 0.001
+        vs = torch.rand(shape[:3], generator=gen, device="cuda") * 0.01 + 0.001
+        kc, vc, q = dev16(w.k_cache), dev16(w.v_cache), dev16(w.q)
+        out = torch.empty_like(q)
+        tables, lens = torch.from_numpy(w.block_tables).cuda(), torch.from_numpy(w.context_lens).cuda()
+        part = args.partition
+        mctx = w.max_blocks_per_seq * sp.block_size
+        ws = torch.empty(max(1, pkv.pkv_decode_workspace_bytes(sp.num_seqs, sp.num_q_heads, sp.num_kv_heads,
+                                                                sp.head_dim, mctx, part)),
+                         dtype=torch.uint8, device="cuda")
+        calls = {
+            "e4m3": lambda: pkv.pkv_decode_attention_e4m3(q, k8, ks, v8, vs, tables, lens, w.scale, out, ws, part),
+            "16bit": lambda: pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part),
+        }
+        ms = {}
+        for name, call in calls.items():
+            for _ in range(args.warmup):
+                call()
+            t0, t1 = ev(), ev()
+            t0.record()
+            for _ in range(args.steps):
+                call()
+            t1.record()
+            torch.cuda.synchronize()
+            assert pkv.pkv_get_last_error() == pkv.PKV_OK
+            ms[name] = t0.elapsed_time(t1) / args.steps
+        nb = algorithmic_bytes(w)
+        ctx = int(w.context_lens.astype(np.int64).sum())
+        kv8 = ctx * 2 * sp.num_kv_heads * (sp.head_dim + 4)
+        bytes8 = kv8 + nb["qo"] + nb["tables"] + nb["lens"]
+        peak = load_peaks()
+        gbs8 = bytes8 / (ms["e4m3"] * 1e-3) / 1e9
+        return {"row": "fp8_kv", "metric": "E4M3 paged decode HBM GB/s (algorithmic bytes / kernel time)",
+                "value": round(gbs8, 1), "unit": "GB/s", "us_per_launch": round(ms["e4m3"] * 1e3, 2),
+                "us_per_launch_16bit": round(ms["16bit"] * 1e3, 2),
+                "speedup_vs_16bit": round(ms["16bit"] / ms["e4m3"], 3),
+                "gbs_16bit": round(nb["total"] / (ms["16bit"] * 1e-3) / 1e9, 1),
+                "peak": peak["hbm_gbs"], "frac": round(gbs8 / peak["hbm_gbs"], 4),
+                "algorithmic_bytes": bytes8, "steps": args.steps, "warmup": args.warmup,
+                "config": {"workload": sp.name, "partition": part, "l2": "working sets > L2 (no flush)",
+                           "kv": "E4M3 codes + fp32 scale per (slot, head) row",
+                           "q_out": workloads.DTYPE_NAMES[sp.dtype]}}
     raise SystemExit(f"unknown row {args.row}")
 
 

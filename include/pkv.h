@@ -62,10 +62,14 @@ typedef enum pkv_status {
     PKV_ERR_SCRATCH_TOO_SMALL = -7 /* the shape needs more scratch than the fixed static area */
 } pkv_status;
 
-typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+/* PKV_E4M3: FP8 E4M3 codes (1 byte) with one fp32 scale per (slot, KV head)
+ * in pkv_cache.scales; used by the *_e4m3 calls only. */
+typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1, PKV_E4M3 = 2 } pkv_dtype;
 
 /* One KV pool: caller-owned device pointer plus its shape [NB][Hkv][bs][D].
- * data must be 16-byte aligned (TMA tiles are read straight from it). */
+ * data must be 16-byte aligned (TMA tiles are read straight from it).
+ * scales: E4M3 pools only, device fp32 [NB][Hkv][bs] (16-byte aligned): the
+ * scale of each cached row; NULL for 16-bit pools. */
 typedef struct pkv_cache {
     void *data;
     pkv_dtype dtype;
@@ -73,6 +77,7 @@ typedef struct pkv_cache {
     int64_t block_size;
     int64_t num_kv_heads;
     int64_t head_dim;
+    float *scales;
 } pkv_cache;
 
 /* A cudaStream_t without including CUDA headers (same underlying type). */
@@ -96,6 +101,38 @@ typedef struct CUstream_st *pkv_stream;
 pkv_status pkv_append(const void *k_new, const void *v_new,
                       const int64_t *slot_mapping, int64_t num_tokens,
                       pkv_cache k_cache, pkv_cache v_cache, pkv_stream stream);
+
+/* --------------------------------------------------------------------------
+ * FP8 E4M3 KV cache.  The pages leave quantization open (adilsher.pro post,
+ * "What I'm Still Figuring Out": how quantization and batching interact);
+ * halving the bytes per token halves the HBM traffic of this path.
+ *
+ * Format: OCP E4M3 codes (no infinities, largest finite 448) with one fp32
+ * scale per cached (token, KV head) row -- a per-row scale keeps each append
+ * a function of its own token (a per-block scale would have to change as
+ * the block fills).  Quantization of a row x[0..D): amax = max |x|, scale =
+ * amax / 448 (1 if amax == 0), code_d = round-to-nearest-even(x_d / scale)
+ * saturated to +-448, both divisions correctly rounded in fp32.  A cached
+ * value is value(code) * scale.
+ *
+ * pkv_append_e4m3: pkv_append into E4M3 pools; k_new / v_new are
+ *   [T][Hkv][D] in new_dtype (PKV_F16 or PKV_BF16).
+ * pkv_decode_attention_e4m3: pkv_decode_attention over E4M3 pools with q and
+ *   out in q_dtype (PKV_F16 or PKV_BF16).  Codes are converted exactly to
+ *   f16 on chip and the products run in f16 with fp32 accumulation (a bf16
+ *   query is converted to f16: exact in f16's normal range); K scales
+ *   multiply the scores, V scales the probabilities.  All partition modes;
+ *   workspace as for pkv_decode_attention.
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_append_e4m3(const void *k_new, const void *v_new, pkv_dtype new_dtype,
+                           const int64_t *slot_mapping, int64_t num_tokens, pkv_cache k_cache,
+                           pkv_cache v_cache, pkv_stream stream);
+pkv_status pkv_decode_attention_e4m3(const void *q, pkv_dtype q_dtype, int64_t num_seqs,
+                                     int64_t num_q_heads, pkv_cache k_cache, pkv_cache v_cache,
+                                     const int32_t *block_tables, int64_t max_blocks_per_seq,
+                                     const int32_t *context_lens, float scale, void *out,
+                                     void *workspace, size_t workspace_bytes,
+                                     int32_t partition_tokens, pkv_stream stream);
 
 /* --------------------------------------------------------------------------
  * pkv_copy_blocks -- device side of copy-on-write: for each (src, dst) pair

@@ -61,6 +61,17 @@ def _bind(lib):
     lib.oracle_prefill_attention.restype = ctypes.c_int
     lib.oracle_prefill_attention.argtypes = [ctypes.c_int, vp, i64, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64,
                                              vp, vp, dbl, vp]
+    lib.oracle_e4m3_value.restype = dbl
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_quantize.restype = ctypes.c_uint8
+    lib.oracle_e4m3_quantize.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_row_scale.restype = ctypes.c_float
+    lib.oracle_e4m3_row_scale.argtypes = [vp, i64, ctypes.c_int]
+    lib.oracle_append_e4m3.restype = ctypes.c_int
+    lib.oracle_append_e4m3.argtypes = [vp, vp, i64, i64, i64, i64, vp, ctypes.c_int, vp, i64]
+    lib.oracle_paged_attention_e4m3.restype = ctypes.c_int
+    lib.oracle_paged_attention_e4m3.argtypes = [ctypes.c_int, vp, i64, i64, vp, vp, vp, vp, i64, i64, i64, i64, vp,
+                                                i64, vp, dbl, vp]
     lib.oracle_copy_blocks.restype = ctypes.c_int
     lib.oracle_copy_blocks.argtypes = [vp, i64, i64, vp, i64]
     lib.oracle_mark_slots.restype = ctypes.c_int
@@ -227,6 +238,43 @@ def prefill_attention(q, k_cache, v_cache, block_tables, query_start, context_le
                                       bt.shape[1], _p(qs), _p(cl), float(scale), _p(out))
     if rc != 0:
         raise ValueError("oracle_prefill_attention: inconsistent lengths or table entry out of range")
+    return out
+
+
+def e4m3_value(code: int, lib=None) -> float:
+    return float((lib or load()).oracle_e4m3_value(code))
+
+
+def e4m3_quantize(y: float, lib=None) -> int:
+    return int((lib or load()).oracle_e4m3_quantize(float(y)))
+
+
+def append_e4m3(cache8: np.ndarray, scales: np.ndarray, new_kv, new_dtype: int, slots, lib=None) -> None:
+    """Quantize rows of new_kv [T][Hkv][D] (16-bit bits) into an E4M3 pool
+    [NB][Hkv][bs][D] (uint8) and its scales [NB][Hkv][bs] (float32), in place."""
+    lib = lib or load()
+    assert cache8.dtype == np.uint8 and scales.dtype == np.float32
+    nb, hkv, bs, d = cache8.shape
+    new = _u16(new_kv)
+    sl = np.ascontiguousarray(slots, dtype=np.int64)
+    rc = lib.oracle_append_e4m3(_p(cache8), _p(scales), nb, hkv, bs, d, _p(new), new_dtype, _p(sl), len(sl))
+    if rc != 0:
+        raise ValueError("oracle_append_e4m3: slot out of range")
+
+
+def attention_e4m3(q, q_dtype, k8, k_scales, v8, v_scales, block_tables, context_lens, scale, lib=None):
+    lib = lib or load()
+    q16 = _u16(q)
+    b, hq, d = q16.shape
+    nb, hkv, bs, _ = k8.shape
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    out = np.zeros((b, hq, d), dtype=np.float64)
+    args = [np.ascontiguousarray(x) for x in (k8, k_scales, v8, v_scales)]
+    rc = lib.oracle_paged_attention_e4m3(q_dtype, _p(q16), b, hq, *(_p(x) for x in args), nb, bs, hkv, d, _p(bt),
+                                         bt.shape[1], _p(cl), float(scale), _p(out))
+    if rc != 0:
+        raise ValueError("oracle_paged_attention_e4m3: invalid arguments")
     return out
 
 

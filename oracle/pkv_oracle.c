@@ -423,3 +423,168 @@ int oracle_prefill_attention(int dtype, const uint16_t *q, int64_t num_tokens,
     }
     return err ? -1 : 0;
 }
+
+/* ---- FP8 E4M3 KV cache -----------------------------------------------------
+ * The pages leave quantization open ("How do quantization and batching
+ * strategy interact?", adilsher.pro post, "What I'm Still Figuring Out").
+ * Format (OCP FP8 E4M3, no infinities): bits s eeee mmm; e = 0: value
+ * m * 2^-9; e >= 1: (1 + m/8) * 2^(e-7); e = 15, m = 7 is NaN; largest
+ * finite 448.  Each appended (token, KV head) row gets one fp32 scale:
+ * scale = amax / 448 (1 if amax == 0), code_d = nearest code to x_d / scale
+ * (ties to the even code, magnitudes past 448 saturate), both divisions in
+ * fp32 with round-to-nearest.  A cached value is value(code) * scale.
+ * Pools: codes [NB][Hkv][bs][D] (bytes), scales [NB][Hkv][bs] (fp32).
+ */
+double oracle_e4m3_value(uint8_t code)
+{
+    int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+uint8_t oracle_e4m3_quantize(float y)
+{
+    /* nearest finite code by exhaustive search over the 127 magnitudes */
+    double a = fabs((double)y);
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7e; ++c) {
+        double err = fabs(oracle_e4m3_value((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    if (a >= 448.0)
+        best = 0x7e;
+    return (uint8_t)(best | (y < 0 ? 0x80 : 0));
+}
+
+float oracle_e4m3_row_scale(const uint16_t *row, int64_t head_dim, int dtype)
+{
+    float amax = 0.0f;
+    for (int64_t d = 0; d < head_dim; ++d) {
+        float x = (float)decode16(dtype, row[d]);
+        if (fabsf(x) > amax)
+            amax = fabsf(x);
+    }
+    return amax > 0.0f ? amax / 448.0f : 1.0f;
+}
+
+int oracle_append_e4m3(uint8_t *cache, float *scales, int64_t num_blocks, int64_t kv_heads,
+                       int64_t block_size, int64_t head_dim, const uint16_t *new_kv,
+                       int new_dtype, const int64_t *slot_mapping, int64_t num_tokens)
+{
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        int64_t block = slot / block_size;
+        int64_t row = slot % block_size;
+        if (block >= num_blocks)
+            return -1;
+        for (int64_t h = 0; h < kv_heads; ++h) {
+            const uint16_t *xrow = new_kv + (t * kv_heads + h) * head_dim;
+            int64_t r = (block * kv_heads + h) * block_size + row;
+            float sc = oracle_e4m3_row_scale(xrow, head_dim, new_dtype);
+            scales[r] = sc;
+            for (int64_t d = 0; d < head_dim; ++d) {
+                float y = (float)decode16(new_dtype, xrow[d]) / sc;
+                cache[r * head_dim + d] = oracle_e4m3_quantize(y);
+            }
+        }
+    }
+    return 0;
+}
+
+static int gather_row_e4m3(const uint8_t *cache, const float *scales, int64_t num_blocks,
+                           int64_t kv_heads, int64_t block_size, int64_t head_dim,
+                           const int32_t *table_row, int64_t pos, int64_t g, double *dst)
+{
+    int64_t phys = table_row[pos / block_size];
+    int64_t row = pos % block_size;
+    if (phys < 0 || phys >= num_blocks)
+        return -1;
+    int64_t r = (phys * kv_heads + g) * block_size + row;
+    for (int64_t d = 0; d < head_dim; ++d)
+        dst[d] = oracle_e4m3_value(cache[r * head_dim + d]) * (double)scales[r];
+    return 0;
+}
+
+/* Decode attention over E4M3 pools: the definition of
+ * oracle_paged_attention with every K/V row dequantized (value * scale). */
+int oracle_paged_attention_e4m3(int q_dtype, const uint16_t *q, int64_t num_seqs,
+                                int64_t num_q_heads, const uint8_t *k_cache, const float *k_scales,
+                                const uint8_t *v_cache, const float *v_scales,
+                                int64_t num_blocks, int64_t block_size, int64_t num_kv_heads,
+                                int64_t head_dim, const int32_t *block_tables,
+                                int64_t max_blocks_per_seq, const int32_t *context_lens,
+                                double scale, double *out)
+{
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+        return -1;
+    int64_t group = num_q_heads / num_kv_heads;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int64_t i = 0; i < num_seqs * num_q_heads; ++i) {
+        int64_t seq = i / num_q_heads, head = i % num_q_heads, g = head / group;
+        int64_t ctx = context_lens[seq];
+        double *o = out + i * head_dim;
+        const int32_t *table_row = block_tables + seq * max_blocks_per_seq;
+        for (int64_t d = 0; d < head_dim; ++d)
+            o[d] = 0.0;
+        if (ctx <= 0)
+            continue;
+        double *qd = malloc(sizeof(double) * head_dim);
+        double *row = malloc(sizeof(double) * head_dim);
+        double *z = malloc(sizeof(double) * ctx);
+        if (!qd || !row || !z) {
+            err |= 1;
+            free(qd);
+            free(row);
+            free(z);
+            continue;
+        }
+        for (int64_t d = 0; d < head_dim; ++d)
+            qd[d] = decode16(q_dtype, q[(seq * num_q_heads + head) * head_dim + d]);
+        double m = -INFINITY;
+        for (int64_t p = 0; p < ctx && !err; ++p) {
+            if (gather_row_e4m3(k_cache, k_scales, num_blocks, num_kv_heads, block_size, head_dim,
+                                table_row, p, g, row)) {
+                err |= 1;
+                break;
+            }
+            double dot = 0.0;
+            for (int64_t d = 0; d < head_dim; ++d)
+                dot += qd[d] * row[d];
+            z[p] = scale * dot;
+            if (z[p] > m)
+                m = z[p];
+        }
+        double l = 0.0;
+        for (int64_t p = 0; p < ctx && !err; ++p) {
+            double w = exp(z[p] - m);
+            l += w;
+            if (gather_row_e4m3(v_cache, v_scales, num_blocks, num_kv_heads, block_size, head_dim,
+                                table_row, p, g, row)) {
+                err |= 1;
+                break;
+            }
+            for (int64_t d = 0; d < head_dim; ++d)
+                o[d] += w * row[d];
+        }
+        if (l > 0.0)
+            for (int64_t d = 0; d < head_dim; ++d)
+                o[d] /= l;
+        free(qd);
+        free(row);
+        free(z);
+    }
+    return err ? -1 : 0;
+}

@@ -28,6 +28,7 @@ PKV_STATIC_SCRATCH_BYTES = 32 << 20
 
 PKV_F16 = 0
 PKV_BF16 = 1
+PKV_E4M3 = 2
 
 PKV_PARTITION_NONE = -1
 PKV_PARTITION_AUTO = 0
@@ -38,7 +39,7 @@ _c_i32, _c_i64, _c_vp, _c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, 
 class pkv_cache(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int), ("num_blocks", ctypes.c_int64),
                 ("block_size", ctypes.c_int64), ("num_kv_heads", ctypes.c_int64),
-                ("head_dim", ctypes.c_int64)]
+                ("head_dim", ctypes.c_int64), ("scales", ctypes.c_void_p)]
 
 
 class pkv_sched_config(ctypes.Structure):
@@ -89,6 +90,10 @@ def _load():
                                                    ctypes.POINTER(_c_i32)]),
         "pkv_seq_append_slots_cow": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp, ctypes.POINTER(_c_i32)]),
         "pkv_copy_blocks": (ctypes.c_int, [pkv_cache, pkv_cache, _c_vp, _c_i64, _c_vp]),
+        "pkv_append_e4m3": (ctypes.c_int, [_c_vp, _c_vp, ctypes.c_int, _c_vp, _c_i64, pkv_cache, pkv_cache, _c_vp]),
+        "pkv_decode_attention_e4m3": (ctypes.c_int, [_c_vp, ctypes.c_int, _c_i64, _c_i64, pkv_cache, pkv_cache,
+                                                     _c_vp, _c_i64, _c_vp, ctypes.c_float, _c_vp, _c_vp, _c_sz,
+                                                     _c_i32, _c_vp]),
         "pkv_sched_create": (ctypes.c_int, [_c_vp, ctypes.POINTER(pkv_sched_config), ctypes.POINTER(_c_vp)]),
         "pkv_sched_destroy": (None, [_c_vp]),
         "pkv_sched_add": (ctypes.c_int, [_c_vp, _c_i64, _c_i32, _c_i32]),
@@ -162,7 +167,19 @@ def cache_desc(cache) -> pkv_cache:
     """Describe a [NB][Hkv][bs][D] fp16/bf16 CUDA tensor as a ``pkv_cache``."""
     _require(cache, "cache", 4)
     nb, hkv, bs, d = cache.shape
-    return pkv_cache(cache.data_ptr(), _dtype_code(cache), nb, bs, hkv, d)
+    return pkv_cache(cache.data_ptr(), _dtype_code(cache), nb, bs, hkv, d, None)
+
+
+def cache_desc_e4m3(codes, scales) -> pkv_cache:
+    """Describe an E4M3 pool: codes uint8 [NB][Hkv][bs][D], scales float32 [NB][Hkv][bs]."""
+    import torch
+
+    _require(codes, "codes", 4)
+    _require(scales, "scales", 3)
+    if codes.dtype != torch.uint8 or scales.dtype != torch.float32 or tuple(scales.shape) != tuple(codes.shape[:3]):
+        raise TypeError("E4M3 pool: uint8 codes [NB][Hkv][bs][D] and float32 scales [NB][Hkv][bs]")
+    nb, hkv, bs, d = codes.shape
+    return pkv_cache(codes.data_ptr(), PKV_E4M3, nb, bs, hkv, d, scales.data_ptr())
 
 
 def pkv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
@@ -286,6 +303,33 @@ def pkv_prefill_attention(q, k_cache, v_cache, block_tables, query_start, contex
                                    context_lens.data_ptr(), float(scale), out.data_ptr(), workspace.data_ptr(),
                                    workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(st, "pkv_prefill_attention")
+
+
+def pkv_append_e4m3(k_new, v_new, slot_mapping, k_codes, k_scales, v_codes, v_scales, stream=None) -> None:
+    """Quantize k_new / v_new [T][Hkv][D] (f16 / bf16) into E4M3 pools at the slots."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (slot_mapping, "slot_mapping")):
+        _require(t, n)
+    st = lib.pkv_append_e4m3(k_new.data_ptr(), v_new.data_ptr(), _dtype_code(k_new), slot_mapping.data_ptr(),
+                             slot_mapping.numel(), cache_desc_e4m3(k_codes, k_scales),
+                             cache_desc_e4m3(v_codes, v_scales), _stream_ptr(stream))
+    _check(st, "pkv_append_e4m3")
+
+
+def pkv_decode_attention_e4m3(q, k_codes, k_scales, v_codes, v_scales, block_tables, context_lens, scale: float,
+                              out, workspace=None, partition_tokens: int = PKV_PARTITION_AUTO, stream=None) -> None:
+    """pkv_decode_attention over E4M3 pools; q / out f16 or bf16."""
+    for t, n in ((q, "q"), (out, "out"), (block_tables, "block_tables"), (context_lens, "context_lens")):
+        _require(t, n)
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        _require(workspace, "workspace")
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = lib.pkv_decode_attention_e4m3(q.data_ptr(), _dtype_code(q), q.shape[0], q.shape[1],
+                                       cache_desc_e4m3(k_codes, k_scales), cache_desc_e4m3(v_codes, v_scales),
+                                       block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+                                       float(scale), out.data_ptr(), ws_ptr or None, ws_bytes,
+                                       int(partition_tokens), _stream_ptr(stream))
+    _check(st, "pkv_decode_attention_e4m3")
 
 
 def pkv_get_last_error() -> int:

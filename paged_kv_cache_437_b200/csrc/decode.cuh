@@ -83,6 +83,8 @@ struct DecodeArgs {
     const int64_t *slots;          // [B], < 0: no append for that sequence
     uint16_t *k_cache, *v_cache;   // the pools, for the generic-store append
     int64_t pool_slots;            // NB * bs
+    // E4M3 pools: one fp32 scale per (slot, KV head), [NB][Hkv][bs]
+    const float *k_scales, *v_scales;
     // chunked prefill: "sequence" s reads block-table row table_rows[s]
     // (several query tokens of one sequence share its row); null = row s
     const int32_t *table_rows;
@@ -94,10 +96,22 @@ struct SmemLayout {
 
 __host__ __device__ inline int align_up_int(int x, int a) { return (x + a - 1) / a * a; }
 
+// Bytes of one pipeline stage: a 16-token K tile and V tile (16-bit), or
+// for the E4M3 cache the 1-byte tiles plus their 16 K and 16 V row scales.
+__host__ __device__ inline int decode_stage_bytes(int D, bool fp8) {
+    return fp8 ? 2 * kTileTokens * D + 2 * kTileTokens * 4 : 2 * kTileTokens * D * 2;
+}
+
+// Per-warp region: its ring of stages and, for E4M3, the 16-bit K and V
+// tiles each stage is converted into (first, 1024-aligned for the swizzle).
+__host__ __device__ inline int decode_warp_bytes(int D, int stages, bool fp8) {
+    const int ring = stages * decode_stage_bytes(D, fp8);
+    return fp8 ? 2 * kTileTokens * D * 2 + align_up_int(ring, 1024) : ring;
+}
+
 __host__ __device__ inline SmemLayout decode_smem_layout(int B, int warps, int stages, int D,
-                                                         bool need_prefix) {
+                                                         bool need_prefix, bool fp8 = false) {
     SmemLayout L;
-    const int tile = kTileTokens * D * 2;
     const int prefix_bytes = need_prefix ? (B + 1) * 4 : 0;
     const int ctx_bytes = need_prefix ? B * 4 : 0;
     L.prefix_off = 0;
@@ -105,7 +119,7 @@ __host__ __device__ inline SmemLayout decode_smem_layout(int B, int warps, int s
     L.bar_off = align_up_int(prefix_bytes + ctx_bytes, 16);
     L.ring_off = align_up_int(L.bar_off + warps * stages * 8, 1024);
     // + 1024: the dynamic smem base is re-aligned to 1024 B at run time
-    L.total = L.ring_off + warps * stages * 2 * tile + 1024;
+    L.total = L.ring_off + warps * decode_warp_bytes(D, stages, fp8) + 1024;
     return L;
 }
 
@@ -254,14 +268,21 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 
 // ------------------------------------------------------------- decode kernel
 
-template <int D, bool BF16, int NT>
+// BF16: q / out are bf16 (else f16).  FP8: the pools hold E4M3 codes with one
+// fp32 scale per (slot, KV head); tiles are converted exactly to f16 in
+// shared memory and the MMAs run in f16 (a bf16 query is converted to f16,
+// exact in f16's normal range); K scales multiply the scores, V scales the
+// probabilities.
+template <int D, bool BF16, int NT, bool FP8 = false>
 __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-    constexpr int kTile = kTileTokens * D * 2;  // bytes of one K (or V) tile
+    constexpr int kTile = kTileTokens * D * 2;  // bytes of one 16-bit K (or V) tile
     constexpr int kMT = D / 16;                 // k-steps of Q K^T == 16-row d tiles of P V
     constexpr int HPU = 8 * NT;                 // query heads per unit (MMA N)
+    constexpr bool MMA_BF16 = FP8 ? false : BF16;
+    constexpr int kStage = FP8 ? 2 * kTileTokens * D + 2 * kTileTokens * 4 : 2 * kTile;
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
@@ -270,13 +291,16 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * warps + warp;
     const bool need_prefix = a.mode != kModeDirect;
-    const SmemLayout L = decode_smem_layout(a.B, warps, a.stages, D, need_prefix);
+    const SmemLayout L = decode_smem_layout(a.B, warps, a.stages, D, need_prefix, FP8);
     int *prefix = reinterpret_cast<int *>(smem_raw + L.prefix_off);
     int *ctxs = reinterpret_cast<int *>(smem_raw + L.ctx_off);
     const uint32_t smem_base = smem_addr(smem_raw);
     const uint32_t bar_base = smem_base + L.bar_off + warp * a.stages * 8;
-    const uint32_t ring_base = ((smem_base + L.ring_off + 1023u) & ~1023u) +
-                               (uint32_t)(warp * a.stages * 2 * kTile);
+    const uint32_t warp_base = ((smem_base + L.ring_off + 1023u) & ~1023u) +
+                               (uint32_t)(warp * decode_warp_bytes(D, a.stages, FP8));
+    // E4M3: the 16-bit conversion tiles come first, the stages after them
+    const uint32_t conv_base = warp_base;
+    const uint32_t ring_base = FP8 ? warp_base + 2 * kTile : warp_base;
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmK);
@@ -439,12 +463,22 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         const int y = (blk * a.Hkv + kvh) * a.bs + row0;
         if (lane == 0) {
             const uint32_t bar = bar_base + stage * 8;
-            const uint32_t kdst = ring_base + stage * 2 * kTile;
-            mbar_arrive_expect_tx(bar, 2 * kTile);
+            const uint32_t kdst = ring_base + stage * kStage;
+            if constexpr (FP8) {
+                // 1-byte tiles (one box of 16 rows x D bytes each) and the
+                // tile's 16 K and 16 V scales (64 contiguous bytes each)
+                mbar_arrive_expect_tx(bar, kStage);
+                tma_load_2d(kdst, &tmK, 0, y, bar);
+                tma_load_2d(kdst + kTileTokens * D, &tmV, 0, y, bar);
+                bulk_load(kdst + 2 * kTileTokens * D, a.k_scales + y, kTileTokens * 4, bar);
+                bulk_load(kdst + 2 * kTileTokens * D + kTileTokens * 4, a.v_scales + y, kTileTokens * 4, bar);
+            } else {
+                mbar_arrive_expect_tx(bar, 2 * kTile);
 #pragma unroll
-            for (int h = 0; h < D / kBoxCols; ++h) {
-                tma_load_2d(kdst + h * kBoxBytes, &tmK, h * kBoxCols, y, bar);
-                tma_load_2d(kdst + kTile + h * kBoxBytes, &tmV, h * kBoxCols, y, bar);
+                for (int h = 0; h < D / kBoxCols; ++h) {
+                    tma_load_2d(kdst + h * kBoxBytes, &tmK, h * kBoxCols, y, bar);
+                    tma_load_2d(kdst + kTile + h * kBoxBytes, &tmV, h * kBoxCols, y, bar);
+                }
             }
         }
         ++issued;
@@ -492,6 +526,15 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             for (int ks = 0; ks < kMT; ++ks) {
                 qb[nt][ks][0] = valid ? __ldg(qr + ks * 8 + c4) : 0u;
                 qb[nt][ks][1] = valid ? __ldg(qr + ks * 8 + 4 + c4) : 0u;
+                if constexpr (FP8 && BF16) {
+                    // the f16 MMA of the E4M3 path: bf16 pairs -> f16 pairs
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const uint32_t w = qb[nt][ks][j];
+                        __half2 h2 = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                        qb[nt][ks][j] = *reinterpret_cast<uint32_t *>(&h2);
+                    }
+                }
             }
         }
 
@@ -513,7 +556,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         // Fused append: this unit holds its sequence's last position.  The
         // new token's row (one 8-byte piece per lane) and slot are loaded here,
         // together with Q, and first used at the last tile.
-        const bool has_new = a.k_new != nullptr && cs.t1 > cs.t0 && cs.t1 * kTileTokens >= cs.ctx;
+        const bool has_new = !FP8 && a.k_new != nullptr && cs.t1 > cs.t0 && cs.t1 * kTileTokens >= cs.ctx;
         int64_t new_slot = -1;
         uint2 kn2 = make_uint2(0, 0), vn2 = make_uint2(0, 0);
         if (has_new) {
@@ -547,9 +590,67 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 break;
             }
             phases ^= 1u << stage;
-            const uint32_t kb = ring_base + stage * 2 * kTile;
-            const uint32_t vb = kb + kTile;
+            uint32_t kb = ring_base + stage * kStage;
+            uint32_t vb = kb + kTile;
             const int nvalid = min(kTileTokens, cs.ctx - t * kTileTokens);
+            float sk_lo = 1.f, sk_hi = 1.f, sv_lo = 1.f, sv_hi = 1.f;
+            if constexpr (FP8) {
+                // convert the E4M3 tiles into this warp's 16-bit tiles in the
+                // 128-byte swizzled layout the ldmatrix addressing expects
+                const uint32_t k8 = kb, v8 = kb + kTileTokens * D, scl = kb + 2 * kTileTokens * D;
+                constexpr int C8 = D / 16;  // 16-byte chunks of codes per row
+#pragma unroll
+                for (int task = lane; task < kTileTokens * C8; task += 32) {
+                    const int r = task / C8, c8 = task - r * C8;
+#pragma unroll
+                    for (int which = 0; which < 2; ++which) {
+                        uint32_t w[4];
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                                     : "r"((which ? v8 : k8) + r * D + c8 * 16));
+                        uint32_t h[8];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            h[2 * j] = e4m3x2_to_f16x2((uint16_t)(w[j] & 0xffffu));
+                            h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(w[j] >> 16));
+                        }
+                        const uint32_t dstb = conv_base + which * kTile;
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const int chunk = 2 * c8 + half;  // 16-byte chunk of the 16-bit row
+                            const uint32_t addr = dstb + (chunk >> 3) * kBoxBytes + r * 128 +
+                                                  ((uint32_t)((chunk & 7) ^ (r & 7)) << 4);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                         "r"(h[4 * half]), "r"(h[4 * half + 1]), "r"(h[4 * half + 2]),
+                                         "r"(h[4 * half + 3])
+                                         : "memory");
+                        }
+                    }
+                }
+                float f[4];
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f[0]) : "r"(scl + g8 * 4));
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f[1]) : "r"(scl + (g8 + 8) * 4));
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f[2]) : "r"(scl + kTileTokens * 4 + g8 * 4));
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f[3]) : "r"(scl + kTileTokens * 4 + (g8 + 8) * 4));
+                sk_lo = f[0];
+                sk_hi = f[1];
+                // a position past the context may hold any scale (even NaN):
+                // its probability is 0 and must stay 0 after the V scale
+                sv_lo = g8 < nvalid ? f[2] : 0.f;
+                sv_hi = g8 + 8 < nvalid ? f[3] : 0.f;
+                __syncwarp();
+                // the codes are converted: the stage goes back to the producer now
+                ++consumed;
+                if (p_has) {
+                    if (lane == 0)
+                        fence_proxy_async_smem();
+                    issue(stage);
+                }
+                if (++stage == a.stages)
+                    stage = 0;
+                kb = conv_base;
+                vb = conv_base + kTile;
+            }
             if (has_new && t == cs.t1 - 1 && new_slot >= 0) {
                 if (new_slot >= a.pool_slots) {
                     if (lane == 0)
@@ -594,7 +695,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 ldmatrix_x4(addr, ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
-                    mma_16816<BF16>(sc[nt], ka, qb[nt][ks][0], qb[nt][ks][1]);
+                    mma_16816<MMA_BF16>(sc[nt], ka, qb[nt][ks][0], qb[nt][ks][1]);
             }
 
             // online softmax per query head (one column of S^T), log2 domain;
@@ -604,10 +705,10 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const float x0 = v_lo ? sc[nt][0] * a.scale_log2 : -INFINITY;
-                const float x1 = v_lo ? sc[nt][1] * a.scale_log2 : -INFINITY;
-                const float x2 = v_hi ? sc[nt][2] * a.scale_log2 : -INFINITY;
-                const float x3 = v_hi ? sc[nt][3] * a.scale_log2 : -INFINITY;
+                const float x0 = v_lo ? sc[nt][0] * (sk_lo * a.scale_log2) : -INFINITY;
+                const float x1 = v_lo ? sc[nt][1] * (sk_lo * a.scale_log2) : -INFINITY;
+                const float x2 = v_hi ? sc[nt][2] * (sk_hi * a.scale_log2) : -INFINITY;
+                const float x3 = v_hi ? sc[nt][3] * (sk_hi * a.scale_log2) : -INFINITY;
                 float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
@@ -631,8 +732,10 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                     o[nt][mt][1] *= al1;
                     o[nt][mt][3] *= al1;
                 }
-                pb[nt][0] = movmatrix_trans(pack2<BF16>(p0, p1));  // tokens 0-7
-                pb[nt][1] = movmatrix_trans(pack2<BF16>(p2, p3));  // tokens 8-15
+                // (E4M3: the V row scales multiply the probabilities here; l
+                // keeps the unscaled sums)
+                pb[nt][0] = movmatrix_trans(pack2<MMA_BF16>(p0 * sv_lo, p1 * sv_lo));  // tokens 0-7
+                pb[nt][1] = movmatrix_trans(pack2<MMA_BF16>(p2 * sv_hi, p3 * sv_hi));  // tokens 8-15
             }
 
             // O^T += V^T P^T.  Positions past the context may hold anything
@@ -657,19 +760,23 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 va[3] &= m23;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
-                    mma_16816<BF16>(o[nt][mt], va, pb[nt][0], pb[nt][1]);
+                    mma_16816<MMA_BF16>(o[nt][mt], va, pb[nt][0], pb[nt][1]);
             }
 
-            // stage consumed: hand it back to the producer for a later tile
-            __syncwarp();
-            ++consumed;
-            if (p_has) {
-                if (lane == 0)
-                    fence_proxy_async_smem();
-                issue(stage);
+            if constexpr (!FP8) {
+                // stage consumed: hand it back to the producer for a later tile
+                __syncwarp();
+                ++consumed;
+                if (p_has) {
+                    if (lane == 0)
+                        fence_proxy_async_smem();
+                    issue(stage);
+                }
+                if (++stage == a.stages)
+                    stage = 0;
+            } else {
+                __syncwarp();  // the conversion tiles are rewritten by the next tile
             }
-            if (++stage == a.stages)
-                stage = 0;
         }
         if (failed)
             break;
@@ -1082,6 +1189,71 @@ __global__ void __launch_bounds__(256) append_kernel(const uint4 *__restrict__ k
         const int64_t dst = ((blk * Hkv + h) * bs + row) * chunks + ch;
         k_cache[dst] = __ldg(k_new + i);
         v_cache[dst] = __ldg(v_new + i);
+    }
+}
+
+// ------------------------------------------------------------- E4M3 append
+
+// One warp per (token, KV head, K|V) row: amax over the row by shuffles,
+// scale = amax / 448 (1 if amax == 0) and y = x / scale as correctly rounded
+// fp32 divisions, codes by round-to-nearest-even with saturation; the codes
+// go to cache[slot / bs][h][slot % bs][:] and the scale beside them.
+template <int D, bool BF16IN>
+__global__ void __launch_bounds__(256) append_e4m3_kernel(const uint16_t *__restrict__ k_new,
+                                                          const uint16_t *__restrict__ v_new,
+                                                          const int64_t *__restrict__ slots, int64_t T, int Hkv,
+                                                          int bs, int64_t nb, uint8_t *__restrict__ k8,
+                                                          float *__restrict__ ks, uint8_t *__restrict__ v8,
+                                                          float *__restrict__ vs, unsigned *err) {
+    constexpr int E = D / 32;  // elements per lane (4 or 2)
+    constexpr unsigned FULL = 0xffffffffu;
+    griddep_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = T * Hkv * 2;
+    for (int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; w < rows;
+         w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int which = (int)(w & 1);  // 0: K, 1: V
+        const int64_t th = w >> 1;       // token * Hkv + head
+        const int64_t t = th / Hkv;
+        const int64_t h = th - t * Hkv;
+        const int64_t slot = __ldg(slots + t);
+        if (slot < 0)
+            continue;
+        const int64_t blk = slot / bs;
+        if (blk >= nb) {
+            if (lane == 0 && which == 0)
+                atomicOr(err, kErrSlot);
+            continue;
+        }
+        const uint16_t *src = (which ? v_new : k_new) + th * D + lane * E;
+        float x[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const uint32_t b = __ldg(src + i);
+            x[i] = BF16IN ? __uint_as_float(b << 16) : __half2float(__ushort_as_half((unsigned short)b));
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < E; ++i)
+            amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+        const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < E; i += 2) {
+            const uint16_t c = f32x2_to_e4m3x2(__fdiv_rn(x[i], scale), __fdiv_rn(x[i + 1], scale));
+            packed |= (uint32_t)c << (8 * i);
+        }
+        const int64_t r = (blk * Hkv + h) * bs + (slot - blk * bs);
+        uint8_t *dst = (which ? v8 : k8) + r * D + lane * E;
+        if constexpr (E == 4)
+            *reinterpret_cast<uint32_t *>(dst) = packed;
+        else
+            *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+        if (lane == 0)
+            (which ? vs : ks)[r] = scale;
     }
 }
 

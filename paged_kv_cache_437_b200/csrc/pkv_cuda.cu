@@ -11,6 +11,7 @@
 #include <algorithm>
 #include <mutex>
 #include <utility>
+#include <tuple>
 #include <vector>
 
 #include "decode.cuh"
@@ -39,6 +40,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool cache_ok(const pkv_cache &c) {
     return c.data && aligned16(c.data) && (c.dtype == PKV_F16 || c.dtype == PKV_BF16) &&
+           c.num_blocks > 0 && c.block_size > 0 && c.num_kv_heads > 0 && c.head_dim > 0;
+}
+
+bool cache_ok_e4m3(const pkv_cache &c) {
+    return c.data && aligned16(c.data) && c.dtype == PKV_E4M3 && c.scales && aligned16(c.scales) &&
            c.num_blocks > 0 && c.block_size > 0 && c.num_kv_heads > 0 && c.head_dim > 0;
 }
 
@@ -125,9 +131,19 @@ bool make_pool_map_uncached(CUtensorMap *map, const pkv_cache &c) {
         return false;
     cuuint64_t dims[2] = {(cuuint64_t)c.head_dim,
                           (cuuint64_t)(c.num_blocks * c.num_kv_heads * c.block_size)};
+    cuuint32_t estr[2] = {1, 1};
+    if (c.dtype == PKV_E4M3) {
+        // E4M3 codes: one box = 16 rows x D bytes, unswizzled (the kernel
+        // reads whole rows and converts them into a swizzled 16-bit tile)
+        cuuint64_t strides[1] = {(cuuint64_t)c.head_dim};
+        cuuint32_t box[2] = {(cuuint32_t)c.head_dim, (cuuint32_t)kTileTokens};
+        CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.data, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        return r == CUDA_SUCCESS;
+    }
     cuuint64_t strides[1] = {(cuuint64_t)c.head_dim * 2};
     cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)kTileTokens};
-    cuuint32_t estr[2] = {1, 1};
     CUtensorMapDataType dt =
         c.dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r = fn(map, dt, 2, c.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -153,17 +169,22 @@ struct Plan {
 using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
 // NT = number of 8-head MMA column tiles per unit: 1 for G <= 8, else 2.
-DecodeKernel pick_decode(int D, bool bf16, int nt) {
-#define PKV_PICK(DD, BB, NN) \
-    if (D == DD && bf16 == BB && nt == NN) return paged_decode_kernel<DD, BB, NN>;
-    PKV_PICK(64, false, 1)
-    PKV_PICK(64, false, 2)
-    PKV_PICK(64, true, 1)
-    PKV_PICK(64, true, 2)
-    PKV_PICK(128, false, 1)
-    PKV_PICK(128, false, 2)
-    PKV_PICK(128, true, 1)
-    PKV_PICK(128, true, 2)
+// bf16: q / out dtype; fp8: E4M3 pools.
+DecodeKernel pick_decode(int D, bool bf16, int nt, bool fp8 = false) {
+#define PKV_PICK(DD, BB, NN, FF) \
+    if (D == DD && bf16 == BB && nt == NN && fp8 == FF) return paged_decode_kernel<DD, BB, NN, FF>;
+#define PKV_PICK_ALL(FF)          \
+    PKV_PICK(64, false, 1, FF)    \
+    PKV_PICK(64, false, 2, FF)    \
+    PKV_PICK(64, true, 1, FF)     \
+    PKV_PICK(64, true, 2, FF)     \
+    PKV_PICK(128, false, 1, FF)   \
+    PKV_PICK(128, false, 2, FF)   \
+    PKV_PICK(128, true, 1, FF)    \
+    PKV_PICK(128, true, 2, FF)
+    PKV_PICK_ALL(false)
+    PKV_PICK_ALL(true)
+#undef PKV_PICK_ALL
 #undef PKV_PICK
     return nullptr;
 }
@@ -192,7 +213,8 @@ cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, s
 // Decide schedule, CTA shape and grid.  PKV_ERR_INVALID if the shape cannot
 // be run (shared memory), PKV_ERR_CUDA if the device cannot be queried.
 pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
-                              int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch);
+                              int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch,
+                              bool fp8);
 
 // Plans depend only on the shape, the device and two tuning variables; they
 // are cached so that a steady decode loop pays no occupancy queries.
@@ -200,23 +222,25 @@ struct PlanKey {
     int dev, warps_env, stages_env;
     int64_t B, Hq, Hkv, D, max_ctx;
     int32_t partition;
-    bool ws, bf16, launch;
+    bool ws, bf16, launch, fp8;
     bool operator==(const PlanKey &o) const {
         return dev == o.dev && warps_env == o.warps_env && stages_env == o.stages_env && B == o.B &&
                Hq == o.Hq && Hkv == o.Hkv && D == o.D && max_ctx == o.max_ctx &&
-               partition == o.partition && ws == o.ws && bf16 == o.bf16 && launch == o.launch;
+               partition == o.partition && ws == o.ws && bf16 == o.bf16 && launch == o.launch &&
+               fp8 == o.fp8;
     }
 };
 
 pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
-                     int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch) {
+                     int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch,
+                     bool fp8 = false) {
     static std::mutex mu;
     static std::vector<std::pair<PlanKey, Plan>> cache;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return PKV_ERR_CUDA;
     const PlanKey key{dev, env_int("PKV_WARPS", 0), env_int("PKV_STAGES", 0), B, Hq, Hkv, D, max_ctx,
-                      partition_tokens, have_workspace, bf16, for_launch};
+                      partition_tokens, have_workspace, bf16, for_launch, fp8};
     {
         std::lock_guard<std::mutex> lock(mu);
         for (auto &e : cache)
@@ -226,7 +250,7 @@ pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int
             }
     }
     pkv_status st = make_plan_uncached(p, B, Hq, Hkv, D, max_ctx, partition_tokens, have_workspace, bf16,
-                                       for_launch);
+                                       for_launch, fp8);
     if (st == PKV_OK) {
         std::lock_guard<std::mutex> lock(mu);
         if (cache.size() >= 64)
@@ -237,7 +261,8 @@ pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int
 }
 
 pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx,
-                              int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch) {
+                              int32_t partition_tokens, bool have_workspace, bool bf16, bool for_launch,
+                              bool fp8) {
     p.Hkv = (int)Hkv;
     p.G = (int)(Hq / Hkv);
     p.nt = p.G > 8 ? 2 : 1;
@@ -272,7 +297,7 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
     if (need_prefix && B * ceil_div64(max_ctx, kTileTokens) * p.npairs >= (int64_t(1) << 31))
         return PKV_ERR_INVALID;
     for (;;) {
-        SmemLayout L = decode_smem_layout((int)B, p.warps, p.stages, (int)D, need_prefix);
+        SmemLayout L = decode_smem_layout((int)B, p.warps, p.stages, (int)D, need_prefix, fp8);
         p.smem = L.total;
         if (p.smem <= kMaxSmemPerCta)
             break;
@@ -288,7 +313,7 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
         return PKV_ERR_CUDA;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int per_sm = 1;
-    DecodeKernel k = pick_decode((int)D, bf16, p.nt);
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8);
     if (!k)
         return PKV_ERR_INVALID;
     // The attribute is per-kernel state shared by every cached plan: set the
@@ -428,11 +453,16 @@ size_t pkv_decode_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t
         return 0;
     if (partition_tokens < 0 || partition_tokens % kTileTokens)
         return 0;
-    Plan p;
-    if (make_plan(p, num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                  partition_tokens, true, false, false) != PKV_OK)
-        return 0;
-    return ws_layout(p, num_seqs, num_q_heads, head_dim, p.max_total_warps).total;
+    // the largest of the layouts a 16-bit or an E4M3 launch of this shape may use
+    size_t best = 0;
+    for (int fp8 = 0; fp8 < 2; ++fp8) {
+        Plan p;
+        if (make_plan(p, num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                      partition_tokens, true, false, false, fp8 != 0) != PKV_OK)
+            return 0;
+        best = std::max(best, ws_layout(p, num_seqs, num_q_heads, head_dim, p.max_total_warps).total);
+    }
+    return best;
 }
 
 }  // extern "C"
@@ -448,11 +478,20 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
                        pkv_cache v_cache, const int32_t *block_tables, int64_t max_blocks_per_seq,
                        const int32_t *context_lens, float scale, void *out, void *workspace,
                        size_t workspace_bytes, int32_t partition_tokens, pkv_stream stream,
-                       const FusedAppend *fa, const int32_t *table_rows = nullptr) {
+                       const FusedAppend *fa, const int32_t *table_rows = nullptr,
+                       pkv_dtype q_dtype = PKV_F16) {
     if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0)
         return PKV_ERR_INVALID;
-    if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
-        return PKV_ERR_INVALID;
+    const bool fp8 = k_cache.dtype == PKV_E4M3;
+    if (fp8) {
+        if (!cache_ok_e4m3(k_cache) || !cache_ok_e4m3(v_cache) || !same_shape(k_cache, v_cache) || fa ||
+            (q_dtype != PKV_F16 && q_dtype != PKV_BF16))
+            return PKV_ERR_INVALID;
+    } else {
+        if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
+            return PKV_ERR_INVALID;
+        q_dtype = k_cache.dtype;
+    }
     const int64_t Hkv = k_cache.num_kv_heads, D = k_cache.head_dim, bs = k_cache.block_size;
     if (num_q_heads % Hkv != 0 || (D != 64 && D != 128) || bs % kTileTokens != 0)
         return PKV_ERR_INVALID;
@@ -473,7 +512,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
         (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
         (reinterpret_cast<uintptr_t>(context_lens) & 3u))
         return PKV_ERR_INVALID;
-    const bool bf16 = k_cache.dtype == PKV_BF16;
+    const bool bf16 = q_dtype == PKV_BF16;
     const int64_t max_ctx = max_blocks_per_seq * bs;
     const bool have_ws = workspace != nullptr;
     if (have_ws && !aligned16(workspace))
@@ -483,10 +522,11 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
 
     Plan p;
     pkv_status ps = make_plan(p, num_seqs, num_q_heads, Hkv, D, max_ctx, partition_tokens, have_ws,
-                              bf16, true);
+                              bf16, true, fp8);
     if (ps == PKV_ERR_INVALID && partition_tokens == PKV_PARTITION_AUTO) {
         // AUTO with a batch too large for the on-chip schedule: one pass per unit
-        ps = make_plan(p, num_seqs, num_q_heads, Hkv, D, max_ctx, PKV_PARTITION_NONE, false, bf16, true);
+        ps = make_plan(p, num_seqs, num_q_heads, Hkv, D, max_ctx, PKV_PARTITION_NONE, false, bf16, true,
+                       fp8);
     }
     if (ps != PKV_OK)
         return ps;
@@ -539,8 +579,10 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.v_cache = static_cast<uint16_t *>(v_cache.data);
     a.pool_slots = k_cache.num_blocks * bs;
     a.table_rows = table_rows;
+    a.k_scales = k_cache.scales;
+    a.v_scales = v_cache.scales;
 
-    DecodeKernel k = pick_decode((int)D, bf16, p.nt);
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8);
     if (!cuda_ok(launch_dependent(k, dim3(p.ctas), dim3(p.warps * 32), p.smem, (cudaStream_t)stream, tmK,
                                   tmV, a)))
         return PKV_ERR_CUDA;
@@ -662,6 +704,59 @@ pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_
     return decode_impl(q, num_tokens, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq, lens,
                        scale, out, workspace_bytes > head ? rest : nullptr, workspace_bytes - head,
                        PKV_PARTITION_AUTO, stream, nullptr, rows);
+}
+
+pkv_status pkv_decode_attention_e4m3(const void *q, pkv_dtype q_dtype, int64_t num_seqs, int64_t num_q_heads,
+                                     pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+                                     int64_t max_blocks_per_seq, const int32_t *context_lens, float scale,
+                                     void *out, void *workspace, size_t workspace_bytes,
+                                     int32_t partition_tokens, pkv_stream stream) {
+    if (k_cache.dtype != PKV_E4M3 || v_cache.dtype != PKV_E4M3)
+        return PKV_ERR_INVALID;
+    return decode_impl(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                       context_lens, scale, out, workspace, workspace_bytes, partition_tokens, stream, nullptr,
+                       nullptr, q_dtype);
+}
+
+pkv_status pkv_append_e4m3(const void *k_new, const void *v_new, pkv_dtype new_dtype,
+                           const int64_t *slot_mapping, int64_t num_tokens, pkv_cache k_cache,
+                           pkv_cache v_cache, pkv_stream stream) {
+    if (num_tokens < 0 || (new_dtype != PKV_F16 && new_dtype != PKV_BF16))
+        return PKV_ERR_INVALID;
+    if (!cache_ok_e4m3(k_cache) || !cache_ok_e4m3(v_cache) || !same_shape(k_cache, v_cache))
+        return PKV_ERR_INVALID;
+    const int64_t D = k_cache.head_dim;
+    if (D != 64 && D != 128)
+        return PKV_ERR_INVALID;
+    if (num_tokens == 0)
+        return PKV_OK;
+    if (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID;
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+    const int64_t rows = num_tokens * k_cache.num_kv_heads * 2;
+    const int64_t blocks = std::min<int64_t>((rows * 32 + 255) / 256, 148 * 16);
+    auto args = std::make_tuple(static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new),
+                                slot_mapping, num_tokens, (int)k_cache.num_kv_heads, (int)k_cache.block_size,
+                                k_cache.num_blocks, static_cast<uint8_t *>(k_cache.data), k_cache.scales,
+                                static_cast<uint8_t *>(v_cache.data), v_cache.scales, err);
+    const bool bf = new_dtype == PKV_BF16;
+    cudaStream_t st = (cudaStream_t)stream;
+    std::apply(
+        [&](auto... xs) {
+            if (D == 128 && bf)
+                append_e4m3_kernel<128, true><<<(unsigned)blocks, 256, 0, st>>>(xs...);
+            else if (D == 128)
+                append_e4m3_kernel<128, false><<<(unsigned)blocks, 256, 0, st>>>(xs...);
+            else if (bf)
+                append_e4m3_kernel<64, true><<<(unsigned)blocks, 256, 0, st>>>(xs...);
+            else
+                append_e4m3_kernel<64, false><<<(unsigned)blocks, 256, 0, st>>>(xs...);
+        },
+        args);
+    return cuda_ok(cudaGetLastError()) ? PKV_OK : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_get_last_error(void) {

@@ -88,6 +88,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a
+// multiple of 16), completion signalled on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -118,6 +127,23 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     uint32_t y;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
     return y;
+}
+
+// ---- FP8 E4M3 conversions ---------------------------------------------------
+
+// Two E4M3 codes (low byte first) -> f16x2 (exact: every E4M3 value is an f16).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+    uint32_t out;
+    asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(codes));
+    return out;
+}
+
+// Two floats -> two E4M3 codes (round to nearest even, saturating to +-448);
+// x0 lands in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float x0, float x1) {
+    uint16_t out;
+    asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(x1), "f"(x0));
+    return out;
 }
 
 // ---- tensor-core MMA m16n8k16, fp32 accumulate ------------------------------

@@ -357,6 +357,65 @@ def check_prefill(lib):
     assert np.array_equal(dec[0], got[qs[1]])
 
 
+def check_e4m3(lib):
+    """E4M3 decode table and quantizer against torch.float8_e4m3fn; append
+    scales and round trips; attention over E4M3 pools against scipy softmax
+    on the dequantized values."""
+    import torch
+
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([lib.oracle_e4m3_value(int(c)) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and np.array_equal(got[~nan], ref[~nan])
+    rng = np.random.default_rng(17)
+    ys = np.concatenate([rng.uniform(-448, 448, 400), rng.standard_normal(400) * 3,
+                         (ref[~nan][:120] + ref[~nan][1:121]) / 2]).astype(np.float32)   # incl. midpoints (ties)
+    ys = ys[np.abs(ys) <= 448]
+    want = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([lib.oracle_e4m3_quantize(float(y)) for y in ys], dtype=np.uint8)
+    assert np.array_equal(mine, want)
+    assert lib.oracle_e4m3_quantize(1000.0) == 0x7e and lib.oracle_e4m3_quantize(-449.0) == 0xfe
+    # append: the largest element becomes +-448, every element within half a step
+    nb, hkv, bs, d = 3, 2, 4, 16
+    pool8 = np.zeros((nb, hkv, bs, d), np.uint8)
+    scales = np.zeros((nb, hkv, bs), np.float32)
+    x = rng.standard_normal((2, hkv, d)).astype(np.float32) * 3
+    bits = f16_bits(x)
+    oracle.append_e4m3(pool8, scales, bits, oracle.F16, np.array([5, 9]), lib=lib)
+    xd = bits_to_f64(bits, oracle.F16)
+    for t, slot in enumerate([5, 9]):
+        blk, row = divmod(slot, bs)
+        for h in range(hkv):
+            sc = np.float32(np.abs(xd[t, h]).max()) / np.float32(448.0)
+            assert scales[blk, h, row] == sc
+            deq = np.array([lib.oracle_e4m3_value(int(c)) for c in pool8[blk, h, row]]) * float(sc)
+            assert np.all(np.abs(deq - xd[t, h]) <= np.abs(xd[t, h]) / 16 + float(sc) * 2 ** -10)
+            assert np.abs(deq).max() == 448.0 * float(sc)
+    # attention over E4M3 pools == scipy softmax on the dequantized rows
+    b, hq, n = 2, 4, 8
+    tables = np.arange(b * n // bs, dtype=np.int32).reshape(b, n // bs)
+    k8 = rng.integers(0, 0x7e, size=(b * n // bs, hkv, bs, d)).astype(np.uint8)
+    v8 = rng.integers(0, 0x7e, size=(b * n // bs, hkv, bs, d)).astype(np.uint8) | 0x80 * (rng.random((b * n // bs, hkv, bs, d)) < 0.5).astype(np.uint8)
+    ks = rng.uniform(0.001, 0.01, size=(b * n // bs, hkv, bs)).astype(np.float32)
+    vs = rng.uniform(0.001, 0.01, size=(b * n // bs, hkv, bs)).astype(np.float32)
+    q = bf16_bits(rng.standard_normal((b, hq, d)))
+    ctx = np.array([8, 5], np.int32)
+    out = oracle.attention_e4m3(q, oracle.BF16, k8, ks, v8, vs, tables, ctx, 0.3, lib=lib)
+    val = np.vectorize(lambda c: lib.oracle_e4m3_value(int(c)))
+    kd = val(k8) * ks[..., None]
+    vd = val(v8) * vs[..., None]
+    qd = bits_to_f64(q, oracle.BF16)
+    for s_ in range(b):
+        for h in range(hq):
+            blocks = tables[s_]
+            kk = np.concatenate([kd[bl, h // 2] for bl in blocks])[:ctx[s_]]
+            vv = np.concatenate([vd[bl, h // 2] for bl in blocks])[:ctx[s_]]
+            p = scipy.special.softmax(0.3 * (kk @ qd[s_, h]))
+            assert np.max(np.abs(out[s_, h] - p @ vv)) < 1e-12
+
+
 ALL_CHECKS = [check_decoders, check_sizing_golden, check_textbook, check_closed_forms, check_gqa_map,
               check_slot_bruteforce, check_append, check_permutation_and_sharing,
-              check_poison_and_scaling, check_split_merge, check_copy_blocks, check_prefill]
+              check_poison_and_scaling, check_split_merge, check_copy_blocks, check_prefill,
+              check_e4m3]

@@ -53,7 +53,7 @@ def _cache(pkv, **kw):
     base = dict(data=0x10000, dtype=pkv.PKV_F16, num_blocks=8, block_size=16, num_kv_heads=2, head_dim=128)
     base.update(kw)
     return pkv.pkv_cache(base["data"], base["dtype"], base["num_blocks"], base["block_size"],
-                         base["num_kv_heads"], base["head_dim"])
+                         base["num_kv_heads"], base["head_dim"], None)
 
 
 @pytest.mark.parametrize("bad", [

@@ -31,6 +31,14 @@ MUTATIONS = {
     "copy_blocks_swapped": ("memmove(cache + dst * block_elems, cache + src * block_elems,",
                             "memmove(cache + src * block_elems, cache + dst * block_elems,"),
     "prefill_window_off_by_one": ("int64_t window = ctx - n + i + 1;", "int64_t window = ctx - n + i;"),
+    "e4m3_bias": ("v = ldexp(1.0 + m / 8.0, e - 7);", "v = ldexp(1.0 + m / 8.0, e - 8);"),
+    "e4m3_ties_odd": ("(err == best_err && (c & 1) == 0 && (best & 1) == 1)",
+                      "(err == best_err && (c & 1) == 1 && (best & 1) == 0)"),
+    "e4m3_scale_range": ("return amax > 0.0f ? amax / 448.0f : 1.0f;", "return amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    "e4m3_gather_block_swapped": ("int64_t phys = table_row[pos / block_size];",
+                                  "int64_t phys = table_row[pos % block_size];"),
+    "e4m3_append_head_transposed": ("const uint16_t *xrow = new_kv + (t * kv_heads + h) * head_dim;",
+                                    "const uint16_t *xrow = new_kv + (h * num_tokens + t) * head_dim;"),
     "kv_sizing_factor": ("return 2 * seq_len * kv_heads * head_dim * dtype_bytes;",
                          "return seq_len * kv_heads * head_dim * dtype_bytes;"),
 }
