@@ -355,6 +355,7 @@ def run_gpu(args, rank, world, local):
             "block_size": sp.block_size,
             "pool_blocks": w.num_blocks,
             "partition": {0: "auto (work-balanced)", -1: "none"}.get(part, f"{part} tokens"),
+            "products": "ffma (CUDA-core variant)" if os.environ.get("PKV_FMA") == "1" else "mma m16n8k16",
             "l2": "flushed between steps" if args.flush_l2 else "per-step KV working set > L2 (no flush)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "step_call": "pkv_append + pkv_decode_attention" if args.unfused else "pkv_append_decode_attention",

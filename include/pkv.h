@@ -181,6 +181,12 @@ pkv_status pkv_copy_blocks(pkv_cache k_cache, pkv_cache v_cache, const int32_t *
  * Results do not depend on which physical blocks hold the data: the order of
  * every reduction is fixed by logical position only.
  * Limits: D in {64, 128}; bs a multiple of 16; Hq % Hkv == 0.
+ *
+ * Tuning variables, read from the environment when a shape is first planned
+ * (plans are cached per shape and per value): PKV_WARPS (warps per CTA,
+ * 1..8), PKV_STAGES (pipeline stages per warp, 2..16), PKV_FMA=1 (16-bit
+ * pools: the two products on the CUDA cores in fp32 FFMA instead of the
+ * tensor-core MMA -- same pipeline and schedules, a measurement aid).
  * ------------------------------------------------------------------------ */
 #define PKV_PARTITION_NONE (-1)
 #define PKV_PARTITION_AUTO 0

@@ -102,15 +102,27 @@ __host__ __device__ inline int decode_stage_bytes(int D, bool fp8) {
     return fp8 ? 2 * kTileTokens * D + 2 * kTileTokens * 4 : 2 * kTileTokens * D * 2;
 }
 
-// Per-warp region: its ring of stages and, for E4M3, the 16-bit K and V
-// tiles each stage is converted into (first, 1024-aligned for the swizzle).
-__host__ __device__ inline int decode_warp_bytes(int D, int stages, bool fp8) {
-    const int ring = stages * decode_stage_bytes(D, fp8);
-    return fp8 ? 2 * kTileTokens * D * 2 + align_up_int(ring, 1024) : ring;
+// Per-warp region (1024-aligned, for the swizzle): its ring of stages; for
+// E4M3 the stages' code tiles come first (2*16*D bytes each, so every tile
+// stays aligned to its swizzle span) and their scales after them.
+// CUDA-core variant: per warp the unit's query rows in fp32 ([8][D + 8], the
+// two column halves 16 bytes apart) and one tile's probabilities ([16][8]).
+__host__ __device__ inline int decode_fma_bytes(int D) { return 8 * (D + 8) * 4 + kTileTokens * 8 * 4; }
+
+__host__ __device__ inline int decode_warp_bytes(int D, int stages, bool fp8, bool fma = false) {
+    return align_up_int(stages * decode_stage_bytes(D, fp8) + (fma ? decode_fma_bytes(D) : 0), 1024);
+}
+
+// Byte offset inside a 16-row E4M3 tile as the TMA wrote it: rows of D bytes
+// with the 16-byte chunks XOR-swizzled by address bits 7.. (128-byte swizzle
+// for D = 128, 64-byte swizzle for D = 64).
+template <int D>
+__device__ __forceinline__ uint32_t e4m3_swz(uint32_t off) {
+    return D == 128 ? off ^ (((off >> 7) & 7u) << 4) : off ^ (((off >> 7) & 3u) << 4);
 }
 
 __host__ __device__ inline SmemLayout decode_smem_layout(int B, int warps, int stages, int D,
-                                                         bool need_prefix, bool fp8 = false) {
+                                                         bool need_prefix, bool fp8 = false, bool fma = false) {
     SmemLayout L;
     const int prefix_bytes = need_prefix ? (B + 1) * 4 : 0;
     const int ctx_bytes = need_prefix ? B * 4 : 0;
@@ -119,7 +131,7 @@ __host__ __device__ inline SmemLayout decode_smem_layout(int B, int warps, int s
     L.bar_off = align_up_int(prefix_bytes + ctx_bytes, 16);
     L.ring_off = align_up_int(L.bar_off + warps * stages * 8, 1024);
     // + 1024: the dynamic smem base is re-aligned to 1024 B at run time
-    L.total = L.ring_off + warps * decode_warp_bytes(D, stages, fp8) + 1024;
+    L.total = L.ring_off + warps * decode_warp_bytes(D, stages, fp8, fma) + 1024;
     return L;
 }
 
@@ -266,6 +278,27 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     }
 }
 
+// Two 16-bit values (low half first) -> two floats (exact).
+template <bool BF16>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+    if constexpr (BF16) {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    } else {
+        __half2 h = *reinterpret_cast<__half2 *>(&w);
+        return __half22float2(h);
+    }
+}
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts_f4(uint32_t addr, float x, float y, float z, float w) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(x), "f"(y), "f"(z), "f"(w) : "memory");
+}
+
 // ------------------------------------------------------------- decode kernel
 
 // BF16: q / out are bf16 (else f16).  FP8: the pools hold E4M3 codes with one
@@ -273,16 +306,20 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 // shared memory and the MMAs run in f16 (a bf16 query is converted to f16,
 // exact in f16's normal range); K scales multiply the scores, V scales the
 // probabilities.
-template <int D, bool BF16, int NT, bool FP8 = false>
+template <int D, bool BF16, int NT, bool FP8 = false, bool FMA = false>
 __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(!FMA || (!FP8 && NT == 1), "the CUDA-core variant: 16-bit pools, 8 heads per unit");
     constexpr int kTile = kTileTokens * D * 2;  // bytes of one 16-bit K (or V) tile
     constexpr int kMT = D / 16;                 // k-steps of Q K^T == 16-row d tiles of P V
     constexpr int HPU = 8 * NT;                 // query heads per unit (MMA N)
     constexpr bool MMA_BF16 = FP8 ? false : BF16;
-    constexpr int kStage = FP8 ? 2 * kTileTokens * D + 2 * kTileTokens * 4 : 2 * kTile;
+    // stage stride: the E4M3 stages hold only the code tiles (scales apart)
+    constexpr int kStage = FP8 ? 2 * kTileTokens * D : 2 * kTile;
+    constexpr int KW8 = FP8 ? D / 16 : 1;  // E4M3: words of one K row a lane reads
+    constexpr int VW8 = FP8 ? D / 32 : 1;  // E4M3: words of one V row a lane reads
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
@@ -291,16 +328,21 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * warps + warp;
     const bool need_prefix = a.mode != kModeDirect;
-    const SmemLayout L = decode_smem_layout(a.B, warps, a.stages, D, need_prefix, FP8);
+    const SmemLayout L = decode_smem_layout(a.B, warps, a.stages, D, need_prefix, FP8, FMA);
     int *prefix = reinterpret_cast<int *>(smem_raw + L.prefix_off);
     int *ctxs = reinterpret_cast<int *>(smem_raw + L.ctx_off);
     const uint32_t smem_base = smem_addr(smem_raw);
     const uint32_t bar_base = smem_base + L.bar_off + warp * a.stages * 8;
     const uint32_t warp_base = ((smem_base + L.ring_off + 1023u) & ~1023u) +
-                               (uint32_t)(warp * decode_warp_bytes(D, a.stages, FP8));
-    // E4M3: the 16-bit conversion tiles come first, the stages after them
-    const uint32_t conv_base = warp_base;
-    const uint32_t ring_base = FP8 ? warp_base + 2 * kTile : warp_base;
+                               (uint32_t)(warp * decode_warp_bytes(D, a.stages, FP8, FMA));
+    const uint32_t ring_base = warp_base;
+    // E4M3: per stage 16 K scales then 16 V scales, after all the code tiles
+    const uint32_t scale_base = ring_base + a.stages * kStage;
+    // CUDA-core variant: query rows and probabilities, after the stages
+    constexpr int kQS = D + 8;  // fp32 row stride of the staged query rows
+    constexpr int FD = D / 32;  // output columns per lane
+    const uint32_t fq_base = ring_base + a.stages * kStage;
+    const uint32_t fp_base = fq_base + 8 * kQS * 4;
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmK);
@@ -465,13 +507,14 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const uint32_t bar = bar_base + stage * 8;
             const uint32_t kdst = ring_base + stage * kStage;
             if constexpr (FP8) {
-                // 1-byte tiles (one box of 16 rows x D bytes each) and the
-                // tile's 16 K and 16 V scales (64 contiguous bytes each)
-                mbar_arrive_expect_tx(bar, kStage);
+                // 1-byte tiles (one swizzled box of 16 rows x D bytes each)
+                // and the tile's 16 K and 16 V scales (64 contiguous bytes each)
+                const uint32_t sdst = scale_base + stage * (4 * kTileTokens * 2);
+                mbar_arrive_expect_tx(bar, kStage + 2 * kTileTokens * 4);
                 tma_load_2d(kdst, &tmK, 0, y, bar);
                 tma_load_2d(kdst + kTileTokens * D, &tmV, 0, y, bar);
-                bulk_load(kdst + 2 * kTileTokens * D, a.k_scales + y, kTileTokens * 4, bar);
-                bulk_load(kdst + 2 * kTileTokens * D + kTileTokens * 4, a.v_scales + y, kTileTokens * 4, bar);
+                bulk_load(sdst, a.k_scales + y, kTileTokens * 4, bar);
+                bulk_load(sdst + kTileTokens * 4, a.v_scales + y, kTileTokens * 4, bar);
             } else {
                 mbar_arrive_expect_tx(bar, 2 * kTile);
 #pragma unroll
@@ -517,15 +560,26 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         // Q^T as the B operand (k = head dim, n = query head)
         uint32_t qb[NT][kMT][2];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+        for (int nt = 0; nt < (FMA ? 0 : NT); ++nt) {
             const int head = nt * 8 + g8;
             const bool valid = head < rows;
             const uint32_t *qr =
                 reinterpret_cast<const uint32_t *>(a.q + ((size_t)cs.seq * a.Hq + h0 + (valid ? head : 0)) * D);
 #pragma unroll
             for (int ks = 0; ks < kMT; ++ks) {
-                qb[nt][ks][0] = valid ? __ldg(qr + ks * 8 + c4) : 0u;
-                qb[nt][ks][1] = valid ? __ldg(qr + ks * 8 + 4 + c4) : 0u;
+                if constexpr (FP8) {
+                    // the E4M3 path takes the head dim in a permuted order
+                    // (the same for K): k-step ks, pair j of lane c4 is
+                    // d = c4 * D/4 + 4 ks + 2 j, +1 -- a dot product does not
+                    // depend on the order of its terms
+                    const uint2 v = valid ? __ldg(reinterpret_cast<const uint2 *>(qr) + (c4 * (D / 16) + ks))
+                                          : make_uint2(0u, 0u);
+                    qb[nt][ks][0] = v.x;
+                    qb[nt][ks][1] = v.y;
+                } else {
+                    qb[nt][ks][0] = valid ? __ldg(qr + ks * 8 + c4) : 0u;
+                    qb[nt][ks][1] = valid ? __ldg(qr + ks * 8 + 4 + c4) : 0u;
+                }
                 if constexpr (FP8 && BF16) {
                     // the f16 MMA of the E4M3 path: bf16 pairs -> f16 pairs
 #pragma unroll
@@ -536,6 +590,24 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                     }
                 }
             }
+        }
+
+        if constexpr (FMA) {
+            // the unit's query rows as fp32 in shared memory (zeros past
+            // `rows`); column c of head h at h * kQS + c (+4 in the upper half)
+            __syncwarp();  // the previous unit is done reading them
+            for (int i = lane; i < D; i += 32) {  // 8 heads x D/8 chunks of 8
+                const int h = i / (D / 8), c = (i - h * (D / 8)) * 8;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (h < rows)
+                    v = __ldg(reinterpret_cast<const uint4 *>(a.q + ((size_t)cs.seq * a.Hq + h0 + h) * D + c));
+                const float2 f0 = unpack2<BF16>(v.x), f1 = unpack2<BF16>(v.y);
+                const float2 f2 = unpack2<BF16>(v.z), f3 = unpack2<BF16>(v.w);
+                const uint32_t dst = fq_base + (uint32_t)(h * kQS + c + (c >= D / 2 ? 4 : 0)) * 4;
+                sts_f4(dst, f0.x, f0.y, f1.x, f1.y);
+                sts_f4(dst + 16, f2.x, f2.y, f3.x, f3.y);
+            }
+            __syncwarp();
         }
 
         {
@@ -570,6 +642,18 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
 
         float o[NT][kMT][4];
         float m_run[NT][2], l_run[NT][2];
+        // CUDA-core variant: heads x this lane's FD columns, per-head state
+        float of[FMA ? 8 : 1][FMA ? FD : 1], mf[FMA ? 8 : 1], lf[FMA ? 8 : 1];
+        if constexpr (FMA) {
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+#pragma unroll
+                for (int j = 0; j < FD; ++j)
+                    of[h][j] = 0.f;
+                mf[h] = -INFINITY;
+                lf[h] = 0.f;
+            }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -594,38 +678,35 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             uint32_t vb = kb + kTile;
             const int nvalid = min(kTileTokens, cs.ctx - t * kTileTokens);
             float sk_lo = 1.f, sk_hi = 1.f, sv_lo = 1.f, sv_hi = 1.f;
+            // E4M3: this lane's code words, taken straight into registers.
+            // K (A operand of S^T, rows = tokens): rows g8 and g8+8, bytes
+            // [c4 D/4, c4 D/4 + D/4) -- word ks is k-step ks of the permuted
+            // head dim.  V (A operand of O^T, rows = head dim): tokens 2c4,
+            // 2c4+1, 2c4+8, 2c4+9, bytes [g8 D/8, g8 D/8 + D/8) -- byte b is
+            // output row d = g8 D/8 + b, i.e. m-tile b/2, row g8 + 8 (b%2).
+            uint32_t kw[2][KW8], vw[4][VW8];
             if constexpr (FP8) {
-                // convert the E4M3 tiles into this warp's 16-bit tiles in the
-                // 128-byte swizzled layout the ldmatrix addressing expects
-                const uint32_t k8 = kb, v8 = kb + kTileTokens * D, scl = kb + 2 * kTileTokens * D;
-                constexpr int C8 = D / 16;  // 16-byte chunks of codes per row
+                const uint32_t k8 = kb, v8 = kb + kTileTokens * D;
+                const uint32_t scl = scale_base + stage * (4 * kTileTokens * 2);
 #pragma unroll
-                for (int task = lane; task < kTileTokens * C8; task += 32) {
-                    const int r = task / C8, c8 = task - r * C8;
+                for (int r = 0; r < 2; ++r) {
 #pragma unroll
-                    for (int which = 0; which < 2; ++which) {
-                        uint32_t w[4];
+                    for (int i = 0; i < KW8 / 4; ++i)
                         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                                     : "r"((which ? v8 : k8) + r * D + c8 * 16));
-                        uint32_t h[8];
+                                     : "=r"(kw[r][4 * i]), "=r"(kw[r][4 * i + 1]), "=r"(kw[r][4 * i + 2]),
+                                       "=r"(kw[r][4 * i + 3])
+                                     : "r"(k8 + e4m3_swz<D>((g8 + 8 * r) * D + c4 * (D / 4) + 16 * i)));
+                }
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            h[2 * j] = e4m3x2_to_f16x2((uint16_t)(w[j] & 0xffffu));
-                            h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(w[j] >> 16));
-                        }
-                        const uint32_t dstb = conv_base + which * kTile;
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const int chunk = 2 * c8 + half;  // 16-byte chunk of the 16-bit row
-                            const uint32_t addr = dstb + (chunk >> 3) * kBoxBytes + r * 128 +
-                                                  ((uint32_t)((chunk & 7) ^ (r & 7)) << 4);
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                         "r"(h[4 * half]), "r"(h[4 * half + 1]), "r"(h[4 * half + 2]),
-                                         "r"(h[4 * half + 3])
-                                         : "memory");
-                        }
-                    }
+                for (int r = 0; r < 4; ++r) {
+                    const int tok = 2 * c4 + (r & 1) + 8 * (r >> 1);
+                    const uint32_t addr = v8 + e4m3_swz<D>(tok * D + g8 * (D / 8));
+                    if constexpr (VW8 == 4)
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(vw[r][0]), "=r"(vw[r][1]), "=r"(vw[r][2]), "=r"(vw[r][3])
+                                     : "r"(addr));
+                    else
+                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(vw[r][0]), "=r"(vw[r][1]) : "r"(addr));
                 }
                 float f[4];
                 asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f[0]) : "r"(scl + g8 * 4));
@@ -639,7 +720,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 sv_lo = g8 < nvalid ? f[2] : 0.f;
                 sv_hi = g8 + 8 < nvalid ? f[3] : 0.f;
                 __syncwarp();
-                // the codes are converted: the stage goes back to the producer now
+                // everything is in registers: the stage goes back to the producer now
                 ++consumed;
                 if (p_has) {
                     if (lane == 0)
@@ -648,8 +729,6 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 }
                 if (++stage == a.stages)
                     stage = 0;
-                kb = conv_base;
-                vb = conv_base + kTile;
             }
             if (has_new && t == cs.t1 - 1 && new_slot >= 0) {
                 if (new_slot >= a.pool_slots) {
@@ -679,90 +758,250 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 __syncwarp();
             }
 
-            // S^T = K Q^T
-            float sc[NT][4];
+            if constexpr (FMA) {
+                // CUDA-core variant.  Scores: lane (token tt, column half hf)
+                // forms the partial dot products of its token's K row half
+                // with every head's query row half; one shuffle adds the halves.
+                const int tt = lane & 15, hf = lane >> 4;
+                float s[8];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                for (int h = 0; h < 8; ++h)
+                    s[h] = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < kMT; ++ks) {
-                const int mi = lane >> 3;
-                const int tok = (lane & 7) + 8 * (mi & 1);
-                const int chunk = 2 * ks + (mi >> 1);
-                const uint32_t addr = kb + (chunk >> 3) * kBoxBytes + tok * 128 +
-                                      ((uint32_t)((chunk & 7) ^ (tok & 7)) << 4);
-                uint32_t ka[4];
-                ldmatrix_x4(addr, ka[0], ka[1], ka[2], ka[3]);
+                for (int c = 0; c < D / 16; ++c) {
+                    const int chunk = hf * (D / 16) + c;  // 16-byte chunk of the K row
+                    uint32_t kw4[4];
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(kw4[0]), "=r"(kw4[1]), "=r"(kw4[2]), "=r"(kw4[3])
+                                 : "r"(kb + (chunk >> 3) * kBoxBytes + tt * 128 +
+                                       ((uint32_t)((chunk & 7) ^ (tt & 7)) << 4)));
+                    float kf[8];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_16816<MMA_BF16>(sc[nt], ka, qb[nt][ks][0], qb[nt][ks][1]);
-            }
-
-            // online softmax per query head (one column of S^T), log2 domain;
-            // this thread holds tokens g8, g8+8 of heads 2*c4, 2*c4+1
-            const bool v_lo = g8 < nvalid;
-            const bool v_hi = g8 + 8 < nvalid;
-            uint32_t pb[NT][2];
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f2 = unpack2<BF16>(kw4[j]);
+                        kf[2 * j] = f2.x;
+                        kf[2 * j + 1] = f2.y;
+                    }
+                    const uint32_t qa = fq_base + (uint32_t)(8 * chunk + 4 * hf) * 4;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float x0 = v_lo ? sc[nt][0] * (sk_lo * a.scale_log2) : -INFINITY;
-                const float x1 = v_lo ? sc[nt][1] * (sk_lo * a.scale_log2) : -INFINITY;
-                const float x2 = v_hi ? sc[nt][2] * (sk_hi * a.scale_log2) : -INFINITY;
-                const float x3 = v_hi ? sc[nt][3] * (sk_hi * a.scale_log2) : -INFINITY;
-                float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+                    for (int h = 0; h < 8; ++h) {
+                        if (h < rows) {
+                            const float4 q0 = lds_f4(qa + h * kQS * 4), q1 = lds_f4(qa + h * kQS * 4 + 16);
+                            float acc = s[h];
+                            acc = fmaf(kf[0], q0.x, acc);
+                            acc = fmaf(kf[1], q0.y, acc);
+                            acc = fmaf(kf[2], q0.z, acc);
+                            acc = fmaf(kf[3], q0.w, acc);
+                            acc = fmaf(kf[4], q1.x, acc);
+                            acc = fmaf(kf[5], q1.y, acc);
+                            acc = fmaf(kf[6], q1.z, acc);
+                            s[h] = fmaf(kf[7], q1.w, acc);
+                        }
+                    }
                 }
-                const float mn0 = fmaxf(m_run[nt][0], mx0);
-                const float mn1 = fmaxf(m_run[nt][1], mx1);
-                const float al0 = exp2f(m_run[nt][0] - mn0);
-                const float al1 = exp2f(m_run[nt][1] - mn1);
-                m_run[nt][0] = mn0;
-                m_run[nt][1] = mn1;
-                const float p0 = exp2f(x0 - mn0), p2 = exp2f(x2 - mn0);
-                const float p1 = exp2f(x1 - mn1), p3 = exp2f(x3 - mn1);
-                l_run[nt][0] = l_run[nt][0] * al0 + (p0 + p2);
-                l_run[nt][1] = l_run[nt][1] * al1 + (p1 + p3);
+                // online softmax per head over the tile's 16 tokens (log2 domain)
+                const bool tv = tt < nvalid;
+                float ph[8];
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    ph[h] = 0.f;
+                    if (h < rows) {
+                        const float sh = s[h] + __shfl_xor_sync(FULL, s[h], 16);
+                        const float x = tv ? sh * a.scale_log2 : -INFINITY;
+                        float mx = x;
+#pragma unroll
+                        for (int off = 1; off < 16; off <<= 1)
+                            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
+                        const float mn = fmaxf(mf[h], mx);
+                        if (mn > mf[h]) {  // uniform: every lane holds the same max
+                            const float al = exp2f(mf[h] - mn);
+                            lf[h] *= al;
+#pragma unroll
+                            for (int j = 0; j < FD; ++j)
+                                of[h][j] *= al;
+                            mf[h] = mn;
+                        }
+                        ph[h] = exp2f(x - mn);
+                        lf[h] += ph[h];
+                    }
+                }
+                if (hf == 0) {
+                    sts_f4(fp_base + tt * 32, ph[0], ph[1], ph[2], ph[3]);
+                    sts_f4(fp_base + tt * 32 + 16, ph[4], ph[5], ph[6], ph[7]);
+                }
+                __syncwarp();
+                // O += P V: lane owns columns [FD lane, FD lane + FD) of every
+                // head; only tokens inside the context are read
+                const int d0 = lane * FD;
+                const int vchunk = d0 >> 3;
+#pragma unroll
+                for (int u = 0; u < kTileTokens; ++u) {
+                    if (u < nvalid) {
+                        const uint32_t addr = vb + (vchunk >> 3) * kBoxBytes + u * 128 +
+                                              ((uint32_t)((vchunk & 7) ^ (u & 7)) << 4) + (uint32_t)(d0 & 7) * 2;
+                        float vf[FD];
+                        if constexpr (FD == 4) {
+                            uint32_t w0, w1;
+                            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(addr));
+                            const float2 v0 = unpack2<BF16>(w0), v1 = unpack2<BF16>(w1);
+                            vf[0] = v0.x;
+                            vf[1] = v0.y;
+                            vf[2 % FD] = v1.x;
+                            vf[3 % FD] = v1.y;
+                        } else {
+                            uint32_t w0;
+                            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(addr));
+                            const float2 v0 = unpack2<BF16>(w0);
+                            vf[0] = v0.x;
+                            vf[1 % FD] = v0.y;
+                        }
+                        const float4 p0 = lds_f4(fp_base + u * 32), p1 = lds_f4(fp_base + u * 32 + 16);
+                        const float pp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            if (h < rows) {
+#pragma unroll
+                                for (int j = 0; j < FD; ++j)
+                                    of[h][j] = fmaf(pp[h], vf[j], of[h][j]);
+                            }
+                        }
+                    }
+                }
+                __syncwarp();  // the probabilities are rewritten by the next tile
+            } else {
+                // S^T = K Q^T, as two independent accumulation chains (even
+                // and odd k-steps) added at the end: half the dependent MMAs
+                float sc[NT][4], sc2[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                    sc2[nt][0] = sc2[nt][1] = sc2[nt][2] = sc2[nt][3] = 0.f;
+                }
+#pragma unroll
+                for (int ks = 0; ks < kMT; ++ks) {
+                    const int mi = lane >> 3;
+                    const int tok = (lane & 7) + 8 * (mi & 1);
+                    const int chunk = 2 * ks + (mi >> 1);
+                    const uint32_t addr = kb + (chunk >> 3) * kBoxBytes + tok * 128 +
+                                          ((uint32_t)((chunk & 7) ^ (tok & 7)) << 4);
+                    uint32_t ka[4];
+                    if constexpr (FP8) {
+                        ka[0] = e4m3x2_to_f16x2((uint16_t)(kw[0][ks] & 0xffffu));
+                        ka[1] = e4m3x2_to_f16x2((uint16_t)(kw[1][ks] & 0xffffu));
+                        ka[2] = e4m3x2_to_f16x2((uint16_t)(kw[0][ks] >> 16));
+                        ka[3] = e4m3x2_to_f16x2((uint16_t)(kw[1][ks] >> 16));
+                    } else {
+                        ldmatrix_x4(addr, ka[0], ka[1], ka[2], ka[3]);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816<MMA_BF16>((ks & 1) ? sc2[nt] : sc[nt], ka, qb[nt][ks][0], qb[nt][ks][1]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        sc[nt][j] += sc2[nt][j];
+                }
+
+                // online softmax per query head (one column of S^T), log2 domain;
+                // this thread holds tokens g8, g8+8 of heads 2*c4, 2*c4+1
+                const bool v_lo = g8 < nvalid;
+                const bool v_hi = g8 + 8 < nvalid;
+                uint32_t pb[NT][2];
+                float x[NT][4];
+                bool up = false;  // some score above its head's running max
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    x[nt][0] = v_lo ? sc[nt][0] * (sk_lo * a.scale_log2) : -INFINITY;
+                    x[nt][1] = v_lo ? sc[nt][1] * (sk_lo * a.scale_log2) : -INFINITY;
+                    x[nt][2] = v_hi ? sc[nt][2] * (sk_hi * a.scale_log2) : -INFINITY;
+                    x[nt][3] = v_hi ? sc[nt][3] * (sk_hi * a.scale_log2) : -INFINITY;
+                    up |= (fmaxf(x[nt][0], x[nt][2]) > m_run[nt][0]) | (fmaxf(x[nt][1], x[nt][3]) > m_run[nt][1]);
+                }
+                // Only when some head's max grows (every first tile, rarely
+                // afterwards) are the maxima reduced across the 8 token rows and
+                // the accumulators rescaled; otherwise the running max stands
+                // and every rescale factor would be exactly 1.
+                if (__any_sync(FULL, up)) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float mx0 = fmaxf(x[nt][0], x[nt][2]), mx1 = fmaxf(x[nt][1], x[nt][3]);
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) {
+                            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+                            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+                        }
+                        const float mn0 = fmaxf(m_run[nt][0], mx0);
+                        const float mn1 = fmaxf(m_run[nt][1], mx1);
+                        const float al0 = exp2f(m_run[nt][0] - mn0);
+                        const float al1 = exp2f(m_run[nt][1] - mn1);
+                        m_run[nt][0] = mn0;
+                        m_run[nt][1] = mn1;
+                        l_run[nt][0] *= al0;
+                        l_run[nt][1] *= al1;
+#pragma unroll
+                        for (int mt = 0; mt < kMT; ++mt) {
+                            o[nt][mt][0] *= al0;
+                            o[nt][mt][2] *= al0;
+                            o[nt][mt][1] *= al1;
+                            o[nt][mt][3] *= al1;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float p0 = exp2f(x[nt][0] - m_run[nt][0]), p2 = exp2f(x[nt][2] - m_run[nt][0]);
+                    const float p1 = exp2f(x[nt][1] - m_run[nt][1]), p3 = exp2f(x[nt][3] - m_run[nt][1]);
+                    l_run[nt][0] += p0 + p2;
+                    l_run[nt][1] += p1 + p3;
+                    // (E4M3: the V row scales multiply the probabilities here; l
+                    // keeps the unscaled sums)
+                    pb[nt][0] = movmatrix_trans(pack2<MMA_BF16>(p0 * sv_lo, p1 * sv_lo));  // tokens 0-7
+                    pb[nt][1] = movmatrix_trans(pack2<MMA_BF16>(p2 * sv_hi, p3 * sv_hi));  // tokens 8-15
+                }
+
+                // O^T += V^T P^T.  Positions past the context may hold anything
+                // (even NaN): zero their V so that 0 * V stays 0 in the MMA.
+                uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
+                if (nvalid < kTileTokens) {
+                    m01 = (2 * c4 < nvalid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < nvalid ? 0xffff0000u : 0u);
+                    m23 = (2 * c4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < nvalid ? 0xffff0000u : 0u);
+                }
 #pragma unroll
                 for (int mt = 0; mt < kMT; ++mt) {
-                    o[nt][mt][0] *= al0;
-                    o[nt][mt][2] *= al0;
-                    o[nt][mt][1] *= al1;
-                    o[nt][mt][3] *= al1;
+                    const int mi = lane >> 3;
+                    const int tok = (lane & 7) + 8 * (mi >> 1);
+                    const int chunk = 2 * mt + (mi & 1);
+                    const uint32_t addr = vb + (chunk >> 3) * kBoxBytes + tok * 128 +
+                                          ((uint32_t)((chunk & 7) ^ (tok & 7)) << 4);
+                    uint32_t va[4];
+                    if constexpr (FP8) {
+                        // pair the codes of two consecutive tokens for one d:
+                        // bytes 2(mt%2) and 2(mt%2)+1 of word mt/2 are rows g8 and g8+8
+                        const int wi = mt >> 1;
+                        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                        const uint32_t p01 = __byte_perm(vw[0][wi], vw[1][wi], sel);
+                        const uint32_t p23 = __byte_perm(vw[2][wi], vw[3][wi], sel);
+                        va[0] = e4m3x2_to_f16x2((uint16_t)(p01 & 0xffffu));
+                        va[1] = e4m3x2_to_f16x2((uint16_t)(p01 >> 16));
+                        va[2] = e4m3x2_to_f16x2((uint16_t)(p23 & 0xffffu));
+                        va[3] = e4m3x2_to_f16x2((uint16_t)(p23 >> 16));
+                    } else {
+                        ldmatrix_x4_trans(addr, va[0], va[1], va[2], va[3]);
+                    }
+                    if (nvalid < kTileTokens) {  // only a ragged tile has positions to mask
+                        va[0] &= m01;
+                        va[1] &= m01;
+                        va[2] &= m23;
+                        va[3] &= m23;
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816<MMA_BF16>(o[nt][mt], va, pb[nt][0], pb[nt][1]);
                 }
-                // (E4M3: the V row scales multiply the probabilities here; l
-                // keeps the unscaled sums)
-                pb[nt][0] = movmatrix_trans(pack2<MMA_BF16>(p0 * sv_lo, p1 * sv_lo));  // tokens 0-7
-                pb[nt][1] = movmatrix_trans(pack2<MMA_BF16>(p2 * sv_hi, p3 * sv_hi));  // tokens 8-15
-            }
 
-            // O^T += V^T P^T.  Positions past the context may hold anything
-            // (even NaN): zero their V so that 0 * V stays 0 in the MMA.
-            uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
-            if (nvalid < kTileTokens) {
-                m01 = (2 * c4 < nvalid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < nvalid ? 0xffff0000u : 0u);
-                m23 = (2 * c4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < nvalid ? 0xffff0000u : 0u);
             }
-#pragma unroll
-            for (int mt = 0; mt < kMT; ++mt) {
-                const int mi = lane >> 3;
-                const int tok = (lane & 7) + 8 * (mi >> 1);
-                const int chunk = 2 * mt + (mi & 1);
-                const uint32_t addr = vb + (chunk >> 3) * kBoxBytes + tok * 128 +
-                                      ((uint32_t)((chunk & 7) ^ (tok & 7)) << 4);
-                uint32_t va[4];
-                ldmatrix_x4_trans(addr, va[0], va[1], va[2], va[3]);
-                va[0] &= m01;
-                va[1] &= m01;
-                va[2] &= m23;
-                va[3] &= m23;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_16816<MMA_BF16>(o[nt][mt], va, pb[nt][0], pb[nt][1]);
-            }
-
             if constexpr (!FP8) {
                 // stage consumed: hand it back to the producer for a later tile
                 __syncwarp();
@@ -774,80 +1013,162 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 }
                 if (++stage == a.stages)
                     stage = 0;
-            } else {
-                __syncwarp();  // the conversion tiles are rewritten by the next tile
             }
         }
         if (failed)
             break;
 
-        // ---- epilogue: per-head sums over the 16 token rows (lanes with the same c4)
+        if constexpr (FMA) {
+            // per-head sums over one column half's 16 token lanes (the other
+            // half holds the same values)
+            const int d0 = lane * FD;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+            for (int h = 0; h < 8; ++h) {
+                if (h < rows) {
+                    float l = lf[h];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1)
-                    l_run[nt][j] += __shfl_xor_sync(FULL, l_run[nt][j], off);
-            }
-        }
-        // Accumulator 8x8 blocks are (d rows) x (head columns); movmatrix
-        // turns each into (head rows) x (d columns): lane (g8, c4) then owns
-        // head g8, d = 16*mt + 8*half + 2*c4 and the next one.
-        if (cs.dest < 0) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float inv0 = l_run[nt][0] > 0.f ? 1.f / l_run[nt][0] : 0.f;
-                const float inv1 = l_run[nt][1] > 0.f ? 1.f / l_run[nt][1] : 0.f;
-                const int head = nt * 8 + g8;
-                uint32_t *dst = reinterpret_cast<uint32_t *>(
-                    a.out + ((size_t)cs.seq * a.Hq + h0 + (head < rows ? head : 0)) * D);
-#pragma unroll
-                for (int mt = 0; mt < kMT; ++mt) {
-                    const uint32_t b0 = movmatrix_trans(pack2<BF16>(o[nt][mt][0] * inv0, o[nt][mt][1] * inv1));
-                    const uint32_t b1 = movmatrix_trans(pack2<BF16>(o[nt][mt][2] * inv0, o[nt][mt][3] * inv1));
-                    if (head < rows) {
-                        dst[mt * 8 + c4] = b0;
-                        dst[mt * 8 + 4 + c4] = b1;
+                    for (int off = 1; off < 16; off <<= 1)
+                        l += __shfl_xor_sync(FULL, l, off);
+                    if (cs.dest < 0) {
+                        const float inv = l > 0.f ? 1.f / l : 0.f;
+                        uint16_t *dst = a.out + ((size_t)cs.seq * a.Hq + h0 + h) * D + d0;
+                        if constexpr (FD == 4)
+                            *reinterpret_cast<uint2 *>(dst) = make_uint2(
+                                pack2<BF16>(of[h][0] * inv, of[h][1 % FD] * inv),
+                                pack2<BF16>(of[h][2 % FD] * inv, of[h][3 % FD] * inv));
+                        else
+                            *reinterpret_cast<uint32_t *>(dst) = pack2<BF16>(of[h][0] * inv, of[h][1 % FD] * inv);
+                    } else {
+                        const size_t row = a.mode == kModePartition
+                                               ? ((size_t)cs.seq * a.Hq + h0 + h) * a.S + cs.dest
+                                               : (size_t)cs.dest * kMaxRows + h;
+                        float *dst = a.part_o + row * D + d0;
+                        if constexpr (FD == 4)
+                            *reinterpret_cast<float4 *>(dst) =
+                                make_float4(of[h][0], of[h][1 % FD], of[h][2 % FD], of[h][3 % FD]);
+                        else
+                            *reinterpret_cast<float2 *>(dst) = make_float2(of[h][0], of[h][1 % FD]);
+                        if (lane == 0) {
+                            a.part_m[row] = mf[h];
+                            a.part_l[row] = l;
+                        }
                     }
                 }
             }
         } else {
+            // ---- epilogue: per-head sums over the 16 token rows (lanes with the same c4)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const int head = nt * 8 + g8;
-                size_t row;
-                if (a.mode == kModePartition)
-                    row = ((size_t)cs.seq * a.Hq + h0 + head) * a.S + cs.dest;
-                else
-                    row = (size_t)cs.dest * kMaxRows + head;
-                float *dst = a.part_o + row * D;
 #pragma unroll
-                for (int mt = 0; mt < kMT; ++mt) {
+                for (int j = 0; j < 2; ++j) {
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        // transpose the fp32 block as two 16-bit halves
-                        const uint32_t xb = __float_as_uint(o[nt][mt][2 * half]);
-                        const uint32_t yb = __float_as_uint(o[nt][mt][2 * half + 1]);
-                        const uint32_t hi = movmatrix_trans((xb >> 16) | (yb & 0xffff0000u));
-                        const uint32_t lo = movmatrix_trans((xb & 0xffffu) | (yb << 16));
-                        const float e0 = __uint_as_float((hi << 16) | (lo & 0xffffu));
-                        const float e1 = __uint_as_float((hi & 0xffff0000u) | (lo >> 16));
-                        if (head < rows)
-                            *reinterpret_cast<float2 *>(dst + mt * 16 + half * 8 + 2 * c4) = make_float2(e0, e1);
-                    }
+                    for (int off = 4; off < 32; off <<= 1)
+                        l_run[nt][j] += __shfl_xor_sync(FULL, l_run[nt][j], off);
                 }
-                // column state: lanes 0-3 hold heads 2*c4, 2*c4+1 of this n-tile
-                if (g8 == 0) {
+            }
+            // Accumulator 8x8 blocks are (d rows) x (head columns); movmatrix
+            // turns each into (head rows) x (d columns): lane (g8, c4) then owns
+            // head g8, d = 16*mt + 8*half + 2*c4 and the next one.
+            if (FP8 && cs.dest < 0) {
+                // permuted head dim: lane (g8, c4) holds heads 2c4, 2c4+1 at
+                // d = g8 D/8 + 2 mt (row g8 of m-tile mt) and d + 1 (row g8+8),
+                // i.e. D/8 consecutive elements of each of its two heads
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const int hc = nt * 8 + 2 * c4 + j;
-                        if (hc < rows) {
-                            const size_t r = a.mode == kModePartition
-                                                 ? ((size_t)cs.seq * a.Hq + h0 + hc) * a.S + cs.dest
-                                                 : (size_t)cs.dest * kMaxRows + hc;
-                            a.part_m[r] = m_run[nt][j];
-                            a.part_l[r] = l_run[nt][j];
+                        const int head = nt * 8 + 2 * c4 + j;
+                        const float inv = l_run[nt][j] > 0.f ? 1.f / l_run[nt][j] : 0.f;
+                        uint32_t wv[kMT];
+#pragma unroll
+                        for (int mt = 0; mt < kMT; ++mt)
+                            wv[mt] = pack2<BF16>(o[nt][mt][j] * inv, o[nt][mt][2 + j] * inv);
+                        if (head < rows) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(a.out + ((size_t)cs.seq * a.Hq + h0 + head) * D +
+                                                                   g8 * (D / 8));
+#pragma unroll
+                            for (int i = 0; i < kMT / 4; ++i)
+                                dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+                        }
+                    }
+                }
+            } else if (FP8) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int head = nt * 8 + 2 * c4 + j;
+                        if (head < rows) {
+                            const size_t row = a.mode == kModePartition
+                                                   ? ((size_t)cs.seq * a.Hq + h0 + head) * a.S + cs.dest
+                                                   : (size_t)cs.dest * kMaxRows + head;
+                            float4 *dst = reinterpret_cast<float4 *>(a.part_o + row * D + g8 * (D / 8));
+#pragma unroll
+                            for (int i = 0; i < kMT / 2; ++i)
+                                dst[i] = make_float4(o[nt][2 * i][j], o[nt][2 * i][2 + j], o[nt][2 * i + 1][j],
+                                                     o[nt][2 * i + 1][2 + j]);
+                            if (g8 == 0) {
+                                a.part_m[row] = m_run[nt][j];
+                                a.part_l[row] = l_run[nt][j];
+                            }
+                        }
+                    }
+                }
+            } else if (cs.dest < 0) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float inv0 = l_run[nt][0] > 0.f ? 1.f / l_run[nt][0] : 0.f;
+                    const float inv1 = l_run[nt][1] > 0.f ? 1.f / l_run[nt][1] : 0.f;
+                    const int head = nt * 8 + g8;
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(
+                        a.out + ((size_t)cs.seq * a.Hq + h0 + (head < rows ? head : 0)) * D);
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        const uint32_t b0 = movmatrix_trans(pack2<BF16>(o[nt][mt][0] * inv0, o[nt][mt][1] * inv1));
+                        const uint32_t b1 = movmatrix_trans(pack2<BF16>(o[nt][mt][2] * inv0, o[nt][mt][3] * inv1));
+                        if (head < rows) {
+                            dst[mt * 8 + c4] = b0;
+                            dst[mt * 8 + 4 + c4] = b1;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int head = nt * 8 + g8;
+                    size_t row;
+                    if (a.mode == kModePartition)
+                        row = ((size_t)cs.seq * a.Hq + h0 + head) * a.S + cs.dest;
+                    else
+                        row = (size_t)cs.dest * kMaxRows + head;
+                    float *dst = a.part_o + row * D;
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            // transpose the fp32 block as two 16-bit halves
+                            const uint32_t xb = __float_as_uint(o[nt][mt][2 * half]);
+                            const uint32_t yb = __float_as_uint(o[nt][mt][2 * half + 1]);
+                            const uint32_t hi = movmatrix_trans((xb >> 16) | (yb & 0xffff0000u));
+                            const uint32_t lo = movmatrix_trans((xb & 0xffffu) | (yb << 16));
+                            const float e0 = __uint_as_float((hi << 16) | (lo & 0xffffu));
+                            const float e1 = __uint_as_float((hi & 0xffff0000u) | (lo >> 16));
+                            if (head < rows)
+                                *reinterpret_cast<float2 *>(dst + mt * 16 + half * 8 + 2 * c4) = make_float2(e0, e1);
+                        }
+                    }
+                    // column state: lanes 0-3 hold heads 2*c4, 2*c4+1 of this n-tile
+                    if (g8 == 0) {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int hc = nt * 8 + 2 * c4 + j;
+                            if (hc < rows) {
+                                const size_t r = a.mode == kModePartition
+                                                     ? ((size_t)cs.seq * a.Hq + h0 + hc) * a.S + cs.dest
+                                                     : (size_t)cs.dest * kMaxRows + hc;
+                                a.part_m[r] = m_run[nt][j];
+                                a.part_l[r] = l_run[nt][j];
+                            }
                         }
                     }
                 }

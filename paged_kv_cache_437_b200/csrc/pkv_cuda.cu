@@ -133,12 +133,14 @@ bool make_pool_map_uncached(CUtensorMap *map, const pkv_cache &c) {
                           (cuuint64_t)(c.num_blocks * c.num_kv_heads * c.block_size)};
     cuuint32_t estr[2] = {1, 1};
     if (c.dtype == PKV_E4M3) {
-        // E4M3 codes: one box = 16 rows x D bytes, unswizzled (the kernel
-        // reads whole rows and converts them into a swizzled 16-bit tile)
+        // E4M3 codes: one box = 16 rows x D bytes, swizzled over the row
+        // width (128-byte swizzle for D = 128, 64-byte for D = 64) so that
+        // the kernel's per-lane row reads are free of bank conflicts
         cuuint64_t strides[1] = {(cuuint64_t)c.head_dim};
         cuuint32_t box[2] = {(cuuint32_t)c.head_dim, (cuuint32_t)kTileTokens};
+        const CUtensorMapSwizzle sw = c.head_dim == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
         CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.data, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         return r == CUDA_SUCCESS;
     }
@@ -164,13 +166,25 @@ struct Plan {
     int smem = 0;
     int Hkv = 0, G = 0, n_hg = 0, npairs = 0;
     int nt = 1, hpu = 8;  // MMA column tiles and query heads per unit
+    bool fma = false;     // CUDA-core variant (PKV_FMA=1, 16-bit pools only)
 };
 
 using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
 // NT = number of 8-head MMA column tiles per unit: 1 for G <= 8, else 2.
-// bf16: q / out dtype; fp8: E4M3 pools.
-DecodeKernel pick_decode(int D, bool bf16, int nt, bool fp8 = false) {
+// bf16: q / out dtype; fp8: E4M3 pools; fma: the CUDA-core variant (16-bit
+// pools, 8 heads per unit), kept to compare against the MMA kernel.
+DecodeKernel pick_decode(int D, bool bf16, int nt, bool fp8 = false, bool fma = false) {
+    if (fma) {
+        if (fp8 || nt != 1)
+            return nullptr;
+        if (D == 64)
+            return bf16 ? paged_decode_kernel<64, true, 1, false, true> : paged_decode_kernel<64, false, 1, false, true>;
+        if (D == 128)
+            return bf16 ? paged_decode_kernel<128, true, 1, false, true>
+                        : paged_decode_kernel<128, false, 1, false, true>;
+        return nullptr;
+    }
 #define PKV_PICK(DD, BB, NN, FF) \
     if (D == DD && bf16 == BB && nt == NN && fp8 == FF) return paged_decode_kernel<DD, BB, NN, FF>;
 #define PKV_PICK_ALL(FF)          \
@@ -219,12 +233,13 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
 // Plans depend only on the shape, the device and two tuning variables; they
 // are cached so that a steady decode loop pays no occupancy queries.
 struct PlanKey {
-    int dev, warps_env, stages_env;
+    int dev, warps_env, stages_env, fma_env;
     int64_t B, Hq, Hkv, D, max_ctx;
     int32_t partition;
     bool ws, bf16, launch, fp8;
     bool operator==(const PlanKey &o) const {
-        return dev == o.dev && warps_env == o.warps_env && stages_env == o.stages_env && B == o.B &&
+        return dev == o.dev && warps_env == o.warps_env && stages_env == o.stages_env &&
+               fma_env == o.fma_env && B == o.B &&
                Hq == o.Hq && Hkv == o.Hkv && D == o.D && max_ctx == o.max_ctx &&
                partition == o.partition && ws == o.ws && bf16 == o.bf16 && launch == o.launch &&
                fp8 == o.fp8;
@@ -239,7 +254,8 @@ pkv_status make_plan(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return PKV_ERR_CUDA;
-    const PlanKey key{dev, env_int("PKV_WARPS", 0), env_int("PKV_STAGES", 0), B, Hq, Hkv, D, max_ctx,
+    const PlanKey key{dev, env_int("PKV_WARPS", 0), env_int("PKV_STAGES", 0), env_int("PKV_FMA", 0),
+                      B, Hq, Hkv, D, max_ctx,
                       partition_tokens, have_workspace, bf16, for_launch, fp8};
     {
         std::lock_guard<std::mutex> lock(mu);
@@ -265,7 +281,10 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
                               bool fp8) {
     p.Hkv = (int)Hkv;
     p.G = (int)(Hq / Hkv);
-    p.nt = p.G > 8 ? 2 : 1;
+    // the CUDA-core variant is a measurement aid for the choice of the MMA
+    // (same pipeline and schedules, FFMA arithmetic); 16-bit pools only
+    p.fma = !fp8 && env_int("PKV_FMA", 0) == 1;
+    p.nt = (p.G > 8 && !p.fma) ? 2 : 1;
     p.hpu = 8 * p.nt;
     p.n_hg = (p.G + p.hpu - 1) / p.hpu;
     p.npairs = (int)Hkv * p.n_hg;
@@ -274,9 +293,12 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
     //    units often and hide that latency best with 12 warps per SM (two
     //    6-warp CTAs);
     //  * otherwise one 8-warp CTA per SM.
-    const int dflt_warps = (partition_tokens <= 0 && B >= 128) ? 6 : 8;
+    //  * E4M3 pools: two 6-warp CTAs per SM everywhere (the conversions
+    //    lengthen each tile's instruction chain; more warps hide it).
+    const int dflt_warps = ((partition_tokens <= 0 && B >= 128) || fp8) ? 6 : 8;
     p.warps = env_int("PKV_WARPS", dflt_warps);
-    p.stages = env_int("PKV_STAGES", 2);
+    // E4M3 stages are half the bytes: twice as many keep as much in flight
+    p.stages = env_int("PKV_STAGES", fp8 ? 4 : 2);
     if (p.warps < 1 || p.warps > 8)
         p.warps = 8;
     if (p.stages < 2 || p.stages > 16)
@@ -297,7 +319,7 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
     if (need_prefix && B * ceil_div64(max_ctx, kTileTokens) * p.npairs >= (int64_t(1) << 31))
         return PKV_ERR_INVALID;
     for (;;) {
-        SmemLayout L = decode_smem_layout((int)B, p.warps, p.stages, (int)D, need_prefix, fp8);
+        SmemLayout L = decode_smem_layout((int)B, p.warps, p.stages, (int)D, need_prefix, fp8, p.fma);
         p.smem = L.total;
         if (p.smem <= kMaxSmemPerCta)
             break;
@@ -313,7 +335,7 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
         return PKV_ERR_CUDA;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int per_sm = 1;
-    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8);
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8, p.fma);
     if (!k)
         return PKV_ERR_INVALID;
     // The attribute is per-kernel state shared by every cached plan: set the
@@ -582,7 +604,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.k_scales = k_cache.scales;
     a.v_scales = v_cache.scales;
 
-    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8);
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8, p.fma);
     if (!cuda_ok(launch_dependent(k, dim3(p.ctas), dim3(p.warps * 32), p.smem, (cudaStream_t)stream, tmK,
                                   tmV, a)))
         return PKV_ERR_CUDA;
