@@ -1203,8 +1203,9 @@ struct MergeArgs {
 // partition mode: S is the bound.
 
 constexpr int kMergeThreads = 128;
-constexpr int kMergeChunk = 512;  // pieces staged in shared memory at a time
+constexpr int kMergeWideThreads = 512;  // one row per CTA, many pieces per row
 
+template <int NTH>
 __device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
     constexpr unsigned FULL = 0xffffffffu;
 #pragma unroll
@@ -1218,7 +1219,7 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) 
     __syncthreads();
     float r = red[0];
 #pragma unroll
-    for (int w = 1; w < kMergeThreads / 32; ++w)
+    for (int w = 1; w < NTH / 32; ++w)
         r = is_max ? fmaxf(r, red[w]) : r + red[w];
     __syncthreads();
     return r;
@@ -1292,10 +1293,13 @@ __device__ __forceinline__ void store_row(const MergeArgs &a, const MergeRow &r,
 
 constexpr int kWarpPieces = 64;  // rows with at most this many pieces: one warp each
 
-// One warp merges one row, kWarpPieces pieces at a time (rescaled online
-// across chunks): lanes hold two pieces' (row, m, l), the reductions are
-// shuffles, every lane owns D/32 consecutive outputs and issues its loads in
-// batches of eight.
+// One warp merges one row, kWarpBatch pieces at a time (rescaled online
+// across batches).  A piece's output row does not depend on its weight, so
+// each batch issues every load at once: lane j < kWarpBatch fetches piece
+// j's (m, l), every lane its D/32 columns of all the batch's outputs; the
+// reductions are shuffles.  One memory round trip per batch.
+constexpr int kWarpBatch = 16;
+
 template <int D, bool BF16>
 __device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRow &r) {
     constexpr unsigned FULL = 0xffffffffu;
@@ -1306,28 +1310,41 @@ __device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRo
 #pragma unroll
     for (int i = 0; i < VEC; ++i)
         acc[i] = 0.f;
-    for (long long k0 = 0; k0 < r.count; k0 += kWarpPieces) {
-        long long rw[2];
-        float mw[2], lw[2];
+    for (long long k0 = 0; k0 < r.count; k0 += kWarpBatch) {
+        const long long kl = k0 + lane;
+        const long long rl = (lane < kWarpBatch && kl < r.count) ? merge_piece(a, r, kl) : -1;
+        const float ml = rl >= 0 ? a.part_m[rl] : -INFINITY;
+        const float ll = rl >= 0 ? a.part_l[rl] : 0.f;
+        float v[kWarpBatch][VEC];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const long long k = k0 + lane + 32 * j;
-            rw[j] = k < r.count ? merge_piece(a, r, k) : -1;
-            mw[j] = rw[j] >= 0 ? a.part_m[rw[j]] : -INFINITY;
-            lw[j] = rw[j] >= 0 ? a.part_l[rw[j]] : 0.f;
+        for (int j = 0; j < kWarpBatch; ++j) {
+            const long long rr = __shfl_sync(FULL, rl, j);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i)
+                v[j][i] = 0.f;
+            if (rr >= 0) {  // an empty piece (-1) has no row
+                const float *p = a.part_o + rr * D + lane * VEC;
+                if constexpr (VEC == 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(p);
+                    v[j][0] = x.x;
+                    v[j][1 % VEC] = x.y;
+                    v[j][2 % VEC] = x.z;
+                    v[j][3 % VEC] = x.w;
+                } else {
+                    const float2 x = *reinterpret_cast<const float2 *>(p);
+                    v[j][0] = x.x;
+                    v[j][1 % VEC] = x.y;
+                }
+            }
         }
-        float cm = fmaxf(mw[0], mw[1]);
+        float cm = ml;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
         const float mnew = fmaxf(M, cm);
         const float rescale = M == -INFINITY ? 0.f : exp2f(M - mnew);
-        float ww[2], lsum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            ww[j] = mw[j] == -INFINITY ? 0.f : exp2f(mw[j] - mnew);
-            lsum += ww[j] * lw[j];
-        }
+        const float w = ml == -INFINITY ? 0.f : exp2f(ml - mnew);
+        float lsum = w * ll;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             lsum += __shfl_xor_sync(FULL, lsum, o);
@@ -1336,26 +1353,12 @@ __device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRo
 #pragma unroll
         for (int i = 0; i < VEC; ++i)
             acc[i] *= rescale;
-        const int n = (int)min((long long)kWarpPieces, r.count - k0);
-#pragma unroll 8
-        for (int k = 0; k < n; ++k) {
-            const int j = k >> 5, src = k & 31;
-            const float w = __shfl_sync(FULL, j ? ww[1] : ww[0], src);
-            const long long rr = __shfl_sync(FULL, j ? rw[1] : rw[0], src);
-            if (w == 0.f)
-                continue;  // an empty piece: its (unwritten) row is never read
-            const float *p = a.part_o + rr * D + lane * VEC;
-            if constexpr (VEC == 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(p);
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-                acc[2] += w * v.z;
-                acc[3] += w * v.w;
-            } else {
-                const float2 v = *reinterpret_cast<const float2 *>(p);
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-            }
+#pragma unroll
+        for (int j = 0; j < kWarpBatch; ++j) {
+            const float wj = __shfl_sync(FULL, w, j);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i)
+                acc[i] = wj != 0.f ? fmaf(wj, v[j][i], acc[i]) : acc[i];
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -1365,59 +1368,70 @@ __device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRo
     store_row<D, BF16>(a, r, lane * VEC, acc, VEC);
 }
 
-// The whole CTA merges one row with many pieces: (row, m, l) staged in shared
-// memory in chunks (rescaled online across chunks), every thread owning one
-// 16-byte column slice and a stride of pieces.
-template <int D, bool BF16>
-__device__ __forceinline__ void merge_row_cta(const MergeArgs &a, const MergeRow &r, float *red,
-                                              long long *s_row, float *s_w, float *s_l, float4 *s_acc) {
+// The whole CTA merges one row with many pieces, GROUPS * kCtaBatch pieces
+// per batch (rescaled online across batches): thread (grp, col) owns one
+// 16-byte column slice of pieces grp, grp + GROUPS, ...; its outputs, and the
+// (m, l) of piece threadIdx.x, are loaded at once, then the weights go
+// through shared memory.
+constexpr int kCtaBatch = 8;
+
+template <int D, bool BF16, int NTH>
+__device__ __forceinline__ void merge_row_cta(const MergeArgs &a, const MergeRow &r, float *red, float *s_w,
+                                              float *s_l, float4 *s_acc) {
     constexpr int COLS = D / 4;
-    constexpr int GROUPS = kMergeThreads / COLS;
+    constexpr int GROUPS = NTH / COLS;
+    constexpr int BATCH = GROUPS * kCtaBatch;  // <= NTH
+    static_assert(BATCH <= NTH, "one (m, l) per thread");
     const int col = threadIdx.x % COLS;
     const int grp = threadIdx.x / COLS;
     float M = -INFINITY, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (long long k0 = 0; k0 < r.count; k0 += kMergeChunk) {
-        const int kn = (int)min((long long)kMergeChunk, r.count - k0);
-        float cmax = -INFINITY;
-        for (int i = threadIdx.x; i < kn; i += kMergeThreads) {
-            const long long rr = merge_piece(a, r, k0 + i);
-            const float m = rr >= 0 ? a.part_m[rr] : -INFINITY;
-            s_l[i] = rr >= 0 ? a.part_l[rr] : 0.f;
-            s_row[i] = rr;
-            s_w[i] = m;
-            cmax = fmaxf(cmax, m);
+    for (long long k0 = 0; k0 < r.count; k0 += BATCH) {
+        const int kn = (int)min((long long)BATCH, r.count - k0);
+        float m = -INFINITY;
+        if (threadIdx.x < kn) {
+            const long long rr = merge_piece(a, r, k0 + threadIdx.x);
+            m = rr >= 0 ? a.part_m[rr] : -INFINITY;
+            s_l[threadIdx.x] = rr >= 0 ? a.part_l[rr] : 0.f;
         }
-        cmax = block_reduce(cmax, true, red);  // also orders the s_* writes
+        float4 v[kCtaBatch];
+#pragma unroll
+        for (int q = 0; q < kCtaBatch; ++q) {
+            const int i = grp + q * GROUPS;
+            const long long rr = i < kn ? merge_piece(a, r, k0 + i) : -1;
+            v[q] = rr >= 0 ? *reinterpret_cast<const float4 *>(a.part_o + rr * D + col * 4)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (threadIdx.x < BATCH)
+            s_w[threadIdx.x] = m;
+        const float cmax = block_reduce<NTH>(m, true, red);  // also orders the s_* writes
         const float mnew = fmaxf(M, cmax);
         const float rescale = M == -INFINITY ? 0.f : exp2f(M - mnew);
         float lsum = 0.f;
-        for (int i = threadIdx.x; i < kn; i += kMergeThreads) {
-            const float m = s_w[i];
+        if (threadIdx.x < kn) {
             const float w = m == -INFINITY ? 0.f : exp2f(m - mnew);
-            s_w[i] = w;
-            lsum += w * s_l[i];
+            s_w[threadIdx.x] = w;
+            lsum = w * s_l[threadIdx.x];
         }
-        lsum = block_reduce(lsum, false, red);
+        lsum = block_reduce<NTH>(lsum, false, red);  // also orders the weights
         L = L * rescale + lsum;
         M = mnew;
         acc.x *= rescale;
         acc.y *= rescale;
         acc.z *= rescale;
         acc.w *= rescale;
-#pragma unroll 8
-        for (int i = grp; i < kn; i += GROUPS) {
-            const float w = s_w[i];
-            if (w == 0.f)
-                continue;  // an empty piece: its (unwritten) row is never read
-            const long long rr = s_row[i];
-            const float4 v = *reinterpret_cast<const float4 *>(a.part_o + rr * D + col * 4);
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
+#pragma unroll
+        for (int q = 0; q < kCtaBatch; ++q) {
+            const int i = grp + q * GROUPS;
+            const float w = i < kn ? s_w[i] : 0.f;
+            if (w != 0.f) {
+                acc.x = fmaf(w, v[q].x, acc.x);
+                acc.y = fmaf(w, v[q].y, acc.y);
+                acc.z = fmaf(w, v[q].z, acc.z);
+                acc.w = fmaf(w, v[q].w, acc.w);
+            }
         }
-        __syncthreads();  // s_row / s_w / s_l are rewritten by the next chunk
+        __syncthreads();  // s_w / s_l are rewritten by the next batch
     }
     s_acc[threadIdx.x] = acc;
     __syncthreads();
@@ -1432,8 +1446,8 @@ __device__ __forceinline__ void merge_row_cta(const MergeArgs &a, const MergeRow
             t.w += u.w;
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
-        const float v[4] = {t.x * inv, t.y * inv, t.z * inv, t.w * inv};
-        store_row<D, BF16>(a, r, threadIdx.x * 4, v, 4);
+        const float vv[4] = {t.x * inv, t.y * inv, t.z * inv, t.w * inv};
+        store_row<D, BF16>(a, r, threadIdx.x * 4, vv, 4);
     }
     __syncthreads();
 }
@@ -1444,18 +1458,19 @@ __device__ __forceinline__ void merge_row_cta(const MergeArgs &a, const MergeRow
 // Pieces with m = -inf (no positions) weigh 0.  Each CTA takes four
 // consecutive (sequence, query head) rows, grid-stride: one warp per row when
 // every row has few pieces, else the four rows one after another with the
-// whole CTA.  The work is latency-bound (a few dependent round trips), so the
-// point is to keep many rows in flight.  Launched as a programmatic
-// dependent of the decode kernel, so its launch overlaps the decode tail.
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergeArgs a) {
-    __shared__ float red[kMergeThreads / 32];
-    __shared__ long long s_row[kMergeChunk];
-    __shared__ float s_w[kMergeChunk];
-    __shared__ float s_l[kMergeChunk];
-    __shared__ float4 s_acc[kMergeThreads];
+// whole CTA.  The work is latency-bound (dependent round trips), so every
+// batch of pieces issues all its loads at once and many rows stay in flight.
+// NTH = 512 (one row per CTA) serves fixed partitions with many pieces per
+// row: 128 pieces per round trip.  Launched as a programmatic dependent of
+// the decode kernel, so its launch overlaps the decode tail.
+template <int D, bool BF16, int NTH = kMergeThreads>
+__global__ void __launch_bounds__(NTH) lse_merge_kernel(const MergeArgs a) {
+    __shared__ float red[NTH / 32];
+    __shared__ float s_w[NTH];
+    __shared__ float s_l[NTH];
+    __shared__ float4 s_acc[NTH];
     griddep_wait();
-    constexpr int ROWS = kMergeThreads / 32;
+    constexpr int ROWS = NTH / 32;
     const int warp = threadIdx.x >> 5;
     const long long rows_total = (long long)a.B * a.Hq;
     const int bound = a.mode == kModePartition ? a.S : a.prefix[a.B + 1];
@@ -1475,7 +1490,7 @@ __global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergeArg
         for (long long row = blockIdx.x; row < rows_total; row += gridDim.x) {
             const MergeRow r = merge_row(a, row);
             if (r.count > 1)
-                merge_row_cta<D, BF16>(a, r, red, s_row, s_w, s_l, s_acc);
+                merge_row_cta<D, BF16, NTH>(a, r, red, s_w, s_l, s_acc);
         }
     }
 }

@@ -634,19 +634,21 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         // enough CTAs for one row each when rows have many pieces; with few
-        // pieces a CTA takes four rows and the rest exit at once
-        const unsigned grid = (unsigned)std::min<int64_t>(num_seqs * num_q_heads, (int64_t)sms * 8);
-        cudaError_t e;
+        // pieces a CTA takes four rows and the rest exit at once.  Fixed
+        // partitions with more pieces per row than one warp's chunk: one
+        // 512-thread CTA per row.
+        const bool wide = p.mode == kModePartition && p.S > kWarpPieces;
+        const int64_t rows = num_seqs * num_q_heads;
+        const unsigned grid = (unsigned)std::min<int64_t>(rows, (int64_t)sms * (wide ? 4 : 8));
+        const dim3 block(wide ? kMergeWideThreads : kMergeThreads);
+        void (*mk)(const MergeArgs) = nullptr;
         if (D == 128)
-            e = bf16 ? launch_dependent(lse_merge_kernel<128, true>, dim3(grid), dim3(kMergeThreads), 0,
-                                        (cudaStream_t)stream, m)
-                     : launch_dependent(lse_merge_kernel<128, false>, dim3(grid), dim3(kMergeThreads), 0,
-                                        (cudaStream_t)stream, m);
+            mk = wide ? (bf16 ? lse_merge_kernel<128, true, kMergeWideThreads> : lse_merge_kernel<128, false, kMergeWideThreads>)
+                      : (bf16 ? lse_merge_kernel<128, true> : lse_merge_kernel<128, false>);
         else
-            e = bf16 ? launch_dependent(lse_merge_kernel<64, true>, dim3(grid), dim3(kMergeThreads), 0,
-                                        (cudaStream_t)stream, m)
-                     : launch_dependent(lse_merge_kernel<64, false>, dim3(grid), dim3(kMergeThreads), 0,
-                                        (cudaStream_t)stream, m);
+            mk = wide ? (bf16 ? lse_merge_kernel<64, true, kMergeWideThreads> : lse_merge_kernel<64, false, kMergeWideThreads>)
+                      : (bf16 ? lse_merge_kernel<64, true> : lse_merge_kernel<64, false>);
+        cudaError_t e = launch_dependent(mk, dim3(grid), block, 0, (cudaStream_t)stream, m);
         if (!cuda_ok(e))
             return PKV_ERR_CUDA;
     }
