@@ -403,8 +403,9 @@ const char *pkv_last_cuda_error(void);
  * come first served -- within max_batch_tokens tokens and max_seqs
  * sequences.  When a request needs a block and none is free, the most
  * recently admitted other request is preempted by recompute (its blocks
- * return to the pool; it rejoins the front of the queue and re-prefills its
- * prompt and generated tokens).  The step's slots come from the allocator,
+ * return to the pool; it rejoins the front of the queue, is readmitted at
+ * the next step at the earliest, and re-prefills its prompt and generated
+ * tokens).  The step's slots come from the allocator,
  * so pkv_batch_tables(seq_ids) gives the matching block tables; run
  * pkv_append with the slots, then pkv_prefill_attention with query_lens as
  * the chunk lengths (a decode token is a chunk of one).  The step that

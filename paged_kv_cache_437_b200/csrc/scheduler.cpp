@@ -17,7 +17,8 @@
 // new block when none is free preempts the most recently admitted running
 // request (recompute: its blocks return to the pool and it goes back to the
 // front of the queue; its prompt and the tokens it had generated are
-// prefilled again when readmitted).  Every sequence's slots come from the
+// prefilled again when readmitted -- at the next step at the earliest, so
+// that the blocks its preemption freed go to the request that needed them).  Every sequence's slots come from the
 // allocator, so the block tables handed to the kernels are exactly its own.
 #include <algorithm>
 #include <cstdint>
@@ -151,6 +152,7 @@ pkv_status pkv_sched_step(void *sched, pkv_sched_batch *out) {
 
     // preempt running request v (recompute): its blocks go back to the pool,
     // it goes back to the front of the queue
+    bool preempted_now = false;  // the queue's front was preempted in this step
     auto preempt = [&](size_t v) {
         for (size_t e = 0; e < plan.size(); ++e) {
             if (plan[e].idx == v) {
@@ -170,6 +172,7 @@ pkv_status pkv_sched_step(void *sched, pkv_sched_batch *out) {
         s->running.erase(s->running.begin() + v);
         in_plan.erase(in_plan.begin() + v);
         s->waiting.push_front(r);
+        preempted_now = true;
         if (out->num_preempted < s->cfg.max_seqs)
             out->preempted_ids[out->num_preempted++] = r.id;
     };
@@ -209,8 +212,9 @@ pkv_status pkv_sched_step(void *sched, pkv_sched_batch *out) {
     }
 
     // 3) admit waiting requests, first come first served; KV memory that is
-    // not there stalls them
-    while (!s->waiting.empty() && budget > 0 && (int32_t)plan.size() < s->cfg.max_seqs &&
+    // not there stalls them, and so does a request preempted in this step
+    // (now at the front of the queue)
+    while (!preempted_now && !s->waiting.empty() && budget > 0 && (int32_t)plan.size() < s->cfg.max_seqs &&
            (int32_t)s->running.size() < s->cfg.max_seqs) {
         Request a = s->waiting.front();
         const int32_t n = std::min({a.target(), s->cfg.chunk_tokens, budget});

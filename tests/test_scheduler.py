@@ -114,3 +114,42 @@ def test_scheduler_argument_checks():
         sched.add(1, 0, 4)
     with pytest.raises(pkv.PkvError):
         sched.add(1, 4, 0)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_configurations_run_to_completion(seed):
+    """Random pools, budgets, chunk sizes and request mixes (some joining
+    mid-run): every step respects its budgets with slots that follow the
+    allocator's tables, every request ends with its prompt and all but its
+    last generated token in the cache, and the pool ends empty."""
+    rng = np.random.default_rng(100 + seed)
+    bs = int(rng.choice([16, 32]))
+    nb = int(rng.integers(16, 96))
+    cap = nb * bs
+    alloc = pkv.BlockAllocator(nb, bs)
+    sched = pkv.Scheduler(alloc, max_batch_tokens=int(rng.integers(64, 1024)), max_seqs=int(rng.integers(2, 24)),
+                          chunk_tokens=int(rng.choice([32, 64, 128, 512])))
+    reqs = {}
+    for rid in range(int(rng.integers(4, 40))):
+        p = int(rng.integers(1, max(2, cap // 3)))
+        m = int(rng.integers(1, max(2, min(64, cap - p))))
+        reqs[rid] = (p, m)
+    late = {rid for rid in reqs if rng.random() < 0.3}
+    for rid, (p, m) in reqs.items():
+        if rid not in late:
+            sched.add(rid, p, m)
+    seen_late = [False]
+
+    def on_step(b):
+        ids = [int(x) for x in b["request_ids"]]
+        assert len(ids) == len(set(ids)), "a request twice in one step"
+        if not seen_late[0]:
+            seen_late[0] = True
+            for rid in sorted(late):
+                sched.add(rid, *reqs[rid])
+
+    _, in_cache, fin = run_to_completion(sched, alloc, max_steps=20_000, on_step=on_step)
+    assert sorted(fin) == sorted(reqs), "every request finishes"
+    for rid, (p, m) in reqs.items():
+        assert in_cache[rid] == p + m - 1, rid
+    assert alloc.num_free() == nb
