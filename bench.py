@@ -84,6 +84,14 @@ def algorithmic_bytes(w) -> dict:
 
 # ------------------------------------------------------------------ helpers
 
+def nvtx(name: str):
+    """An NVTX range around one phase of the run (visible to a system
+    profiler), never inside a per-step loop."""
+    import torch
+
+    return torch.cuda.nvtx.range(name)
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -275,9 +283,10 @@ def run_gpu(args, rank, world, local):
     pkv.pkv_append(kn, vn, slots, kc, vc, stream)
     pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
     pkv.pkv_append_decode_attention(kn, vn, slots, q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
+    with nvtx("pkv warm-up"):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
     if pkv.pkv_get_last_error() != pkv.PKV_OK:
         raise RuntimeError("device check failed during warm-up")
 
@@ -288,27 +297,29 @@ def run_gpu(args, rank, world, local):
         # K whole steps, events only around the region (no events between the
         # kernels, so each launch can overlap the previous kernel's tail)
         t0, t1 = ev(), ev()
-        t0.record(stream)
-        for i in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize()
+        with nvtx("pkv timed steps"):
+            t0.record(stream)
+            for i in range(args.steps):
+                if flush is not None:
+                    flush.zero_()
+                step()
+            t1.record(stream)
+            torch.cuda.synchronize()
         barrier()
         step_ms = t0.elapsed_time(t1)
         # the dominant kernel: K launches of the decode kernel (the fused
         # append + decode call of the step, or the decode call alone) back to
         # back, plus its merge when contexts are split
         d0, d1 = ev(), ev()
-        d0.record(stream)
-        for i in range(args.steps):
-            if args.unfused:
-                c_decode(*decode_args)
-            else:
-                c_fused(*fused_args)
-        d1.record(stream)
-        torch.cuda.synchronize()
+        with nvtx("pkv dominant kernel"):
+            d0.record(stream)
+            for i in range(args.steps):
+                if args.unfused:
+                    c_decode(*decode_args)
+                else:
+                    c_fused(*fused_args)
+            d1.record(stream)
+            torch.cuda.synchronize()
     barrier()
     dec_ms = d0.elapsed_time(d1) / args.steps
     if flush is not None:
@@ -325,7 +336,8 @@ def run_gpu(args, rank, world, local):
         raise RuntimeError("device check failed in the timed region")
 
     # ---- end to end through the C ABI with host buffers
-    e2e = None if args.no_e2e else measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out)
+    with nvtx("pkv end-to-end"):
+        e2e = None if args.no_e2e else measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out)
     peaks = load_peaks()
     ms_per_step = max_ms / args.steps
     value = weak_scaling_value(nb_bytes["total"], world, args.steps, max_ms)
