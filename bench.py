@@ -2,13 +2,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--partition P] [--flush-l2] [--impl reference]
+    python bench.py --row cow|prefill|sched|fp8 [--workload NAME]
 
 A step is the whole hot path on one batch: the append of every sequence's new
 token and the attention (decode kernel + log-sum-exp merge when the schedule
 splits contexts), by default through the fused pkv_append_decode_attention
-call (``--unfused``: pkv_append then pkv_decode_attention).  Inputs are synthetic and seeded (``workloads``),
-shaped like the pages' examples; the default workload is the 13B-shaped layer
-(32 sequences x 2048 context, 40/40 heads, D 128, block 16, fp16).
+call (``--unfused``: pkv_append then pkv_decode_attention).  Inputs are
+synthetic and seeded (``workloads``), shaped like the pages' examples; the
+default workload is the 13B-shaped layer (32 sequences x 2048 context, 40/40
+heads, D 128, block 16, fp16).  ``--row`` measures one of the rows next to
+the hot path instead (copy-on-write block copies, chunked prefill, the host
+scheduler, E4M3 decode) and prints one JSON line tagged "row".
 
 Metric: achieved HBM GB/s of algorithmic bytes (KV read for every sequence's
 context + Q + O + used block-table entries + context lengths) per step time,
