@@ -132,3 +132,18 @@ def test_workspace_query_without_gpu_is_zero_or_sized():
     assert pkv.pkv_decode_workspace_bytes(4, 8, 2, 128, 4096, pkv.PKV_PARTITION_NONE) == 0
     assert pkv.pkv_decode_workspace_bytes(4, 8, 2, 96, 4096, 512) == 0      # bad head_dim
     assert pkv.pkv_decode_workspace_bytes(4, 8, 3, 128, 4096, 512) == 0     # Hq % Hkv
+
+
+def test_binding_without_the_library_fails_loudly(tmp_path):
+    """No CPU fallback: a copy of the package without libpkv.so refuses to import."""
+    import shutil
+    import subprocess
+    import sys
+
+    src = os.path.join(ROOT, "paged_kv_cache_437_b200")
+    dst = tmp_path / "paged_kv_cache_437_b200"
+    shutil.copytree(src, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import paged_kv_cache_437_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "not built" in r.stderr
