@@ -206,9 +206,8 @@ def pkv_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: in
                                               max_context_len, partition_tokens))
 
 
-def pkv_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
-                         workspace=None, partition_tokens: int = PKV_PARTITION_AUTO, stream=None) -> None:
-    """out[B][Hq][D] = paged decode attention of q[B][Hq][D] over the caches."""
+def _check_decode_args(q, k_cache, block_tables, context_lens, out) -> None:
+    """Dtype and shape checks shared by the decode wrappers."""
     import torch
 
     for t, n in ((q, "q"), (out, "out"), (block_tables, "block_tables"), (context_lens, "context_lens")):
@@ -220,6 +219,12 @@ def pkv_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale:
     if q.dim() != 3 or out.shape != q.shape or block_tables.dim() != 2 or \
             block_tables.shape[0] != q.shape[0] or context_lens.numel() != q.shape[0]:
         raise ValueError("shapes: q/out [B][Hq][D], block_tables [B][MB], context_lens [B]")
+
+
+def pkv_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                         workspace=None, partition_tokens: int = PKV_PARTITION_AUTO, stream=None) -> None:
+    """out[B][Hq][D] = paged decode attention of q[B][Hq][D] over the caches."""
+    _check_decode_args(q, k_cache, block_tables, context_lens, out)
     ws_ptr, ws_bytes = 0, 0
     if workspace is not None:
         _require(workspace, "workspace")
@@ -241,8 +246,7 @@ def pkv_decode_attention_static_scratch(q, k_cache, v_cache, block_tables, conte
     """pkv_decode_attention for callers that cannot allocate device memory:
     the split scratch is the library's fixed device array (see include/pkv.h).
     Calls that overlap on the GPU share that array and must be serialised."""
-    for t, n in ((q, "q"), (out, "out"), (block_tables, "block_tables"), (context_lens, "context_lens")):
-        _require(t, n)
+    _check_decode_args(q, k_cache, block_tables, context_lens, out)
     st = lib.pkv_decode_attention_static_scratch(q.data_ptr(), q.shape[0], q.shape[1], cache_desc(k_cache),
                                                  cache_desc(v_cache), block_tables.data_ptr(),
                                                  block_tables.shape[1], context_lens.data_ptr(), float(scale),

@@ -870,8 +870,16 @@ extern "C" pkv_status pkv_decode_attention_static_scratch(
     const size_t need = pkv_decode_workspace_bytes(
         num_seqs, num_q_heads, k_cache.num_kv_heads, k_cache.head_dim,
         max_blocks_per_seq * k_cache.block_size, partition_tokens);
-    if (need == 0)
+    if (need == 0) {
+        // AUTO on a batch too large for the on-chip schedule: the regular
+        // entry point then runs one pass per unit with no scratch at all, and
+        // so does this one (an invalid shape is refused there just the same)
+        if (partition_tokens == PKV_PARTITION_AUTO)
+            return pkv_decode_attention(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables,
+                                        max_blocks_per_seq, context_lens, scale, out, nullptr, 0,
+                                        partition_tokens, stream);
         return PKV_ERR_INVALID;  // shape rejected (or no device to size it on)
+    }
     if (need > (size_t)PKV_STATIC_SCRATCH_BYTES)
         return PKV_ERR_SCRATCH_TOO_SMALL;
     void *scratch = static_scratch_device_ptr();

@@ -222,6 +222,39 @@ def check_slot_bruteforce(lib):
             assert oracle.slot_of(tables[s], p, bs, lib=lib) == slot
 
 
+def check_slot_mask(lib):
+    """The attended-slot mask (which slots every GPU test leaves un-poisoned)
+    against a brute-force enumeration: walk each sequence's table block by
+    block and row by row, counting positions, and keep the first lens[s].
+    Lengths 0, 1, bs, bs + 1 and a full table; two sequences share blocks."""
+    rng = np.random.default_rng(11)
+    bs, mb, nb = 4, 5, 40
+    lens = np.array([0, 1, bs, bs + 1, mb * bs, 7, 13], np.int32)
+    b = lens.size
+    tables = np.full((b, mb), -1, np.int32)
+    free = list(rng.permutation(nb))
+    for s in range(b):
+        need = -(-int(lens[s]) // bs)
+        for j in range(need):
+            tables[s, j] = free.pop()
+    tables[6, :2] = tables[4, :2]          # a shared two-block prefix
+    expected = np.zeros(nb * bs, bool)
+    for s in range(b):
+        pos = 0
+        for blk in tables[s]:
+            for r in range(bs):
+                if pos < lens[s]:
+                    expected[int(blk) * bs + r] = True
+                pos += 1
+    got = oracle.slot_mask(tables, lens, bs, nb, lib=lib)
+    assert got.shape == expected.shape and np.array_equal(got, expected)
+    # the mask of the lengths before one append leaves exactly the new slots out
+    prior = np.maximum(lens - 1, 0)
+    got_prior = oracle.slot_mask(tables, prior, bs, nb, lib=lib)
+    new_slots = {int(tables[s, (lens[s] - 1) // bs]) * bs + int(lens[s] - 1) % bs for s in range(b) if lens[s] > 0}
+    assert set(np.nonzero(got & ~got_prior)[0].tolist()) == new_slots - set(np.nonzero(got_prior)[0].tolist())
+
+
 def check_append(lib, dtype=oracle.F16):
     rng = np.random.default_rng(9)
     nb, hkv, bs, d, t = 6, 3, 4, 8, 7
@@ -416,6 +449,6 @@ def check_e4m3(lib):
 
 
 ALL_CHECKS = [check_decoders, check_sizing_golden, check_textbook, check_closed_forms, check_gqa_map,
-              check_slot_bruteforce, check_append, check_permutation_and_sharing,
+              check_slot_bruteforce, check_slot_mask, check_append, check_permutation_and_sharing,
               check_poison_and_scaling, check_split_merge, check_copy_blocks, check_prefill,
               check_e4m3]

@@ -39,6 +39,12 @@ MUTATIONS = {
                                   "int64_t phys = table_row[pos % block_size];"),
     "e4m3_append_head_transposed": ("const uint16_t *xrow = new_kv + (t * kv_heads + h) * head_dim;",
                                     "const uint16_t *xrow = new_kv + (h * num_tokens + t) * head_dim;"),
+    "slot_mask_last_position_dropped": ("for (int64_t p = 0; p < lens[s]; ++p) {",
+                                        "for (int64_t p = 0; p + 1 < lens[s]; ++p) {"),
+    "slot_mask_whole_blocks": ("mask[b * block_size + p % block_size] = 1;",
+                               "for (int64_t r = 0; r < block_size; ++r) mask[b * block_size + r] = 1;"),
+    "slot_mask_row_from_block": ("mask[b * block_size + p % block_size] = 1;",
+                                 "mask[b * block_size + p / block_size] = 1;"),
     "kv_sizing_factor": ("return 2 * seq_len * kv_heads * head_dim * dtype_bytes;",
                          "return seq_len * kv_heads * head_dim * dtype_bytes;"),
 }

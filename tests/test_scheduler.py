@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 
-pkv = pytest.importorskip("paged_kv_cache_437_b200")
+import paged_kv_cache_437_b200 as pkv  # a missing library fails here, never skips
 
 
 def run_to_completion(sched, alloc, max_steps=10_000, check_slots=True, on_step=None):
