@@ -53,7 +53,7 @@ METRIC = "paged decode attention: achieved HBM GB/s (% of B200 peak); decode tok
 DEFAULT_WORKLOAD = "llama13b"
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_437_b200", "csrc", f)
-                  for f in ("decode.cuh", "ptx.cuh", "pkv_cuda.cu")]
+                  for f in ("decode.cuh", "mq_attention.cuh", "ptx.cuh", "pkv_cuda.cu")]
 
 
 # ------------------------------------------------------------------ bytes
@@ -101,8 +101,11 @@ def load_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
-    return dict(hbm_gbs=6650.0, source="fallback")
+        out = dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
+        if "bf16_tflops" in d:
+            out["bf16_tflops"] = float(d["bf16_tflops"])
+        return out
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
 
 
 def kernel_hash() -> str:
@@ -275,13 +278,22 @@ def run_gpu(args, rank, world, local):
     c_fused = pkv.lib.pkv_append_decode_attention
     fused_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr()) + decode_args
 
-    if args.unfused:
-        def step():
-            c_append(*append_args)
-            c_decode(*decode_args)
-    else:
-        def step():
-            c_fused(*fused_args)
+    def make_step(q, kn, vn, slots, tables, lens):
+        """The step's raw C ABI calls on these device inputs."""
+        a_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr(), slots.numel(), kdesc, vdesc, sptr)
+        d_args = (q.data_ptr(), q.shape[0], q.shape[1], kdesc, vdesc, tables.data_ptr(), tables.shape[1],
+                  lens.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, part, sptr)
+        f_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr()) + d_args
+        if args.unfused:
+            def step():
+                c_append(*a_args)
+                c_decode(*d_args)
+        else:
+            def step():
+                c_fused(*f_args)
+        return step
+
+    step = make_step(q, kn, vn, slots, tables, lens)
 
     # the binding path once, with its argument checks
     pkv.pkv_append(kn, vn, slots, kc, vc, stream)
@@ -341,7 +353,7 @@ def run_gpu(args, rank, world, local):
 
     # ---- end to end through the C ABI with host buffers
     with nvtx("pkv end-to-end"):
-        e2e = None if args.no_e2e else measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out)
+        e2e = None if args.no_e2e else measure_e2e(args, make_step, stream, q, kn, vn, slots, tables, lens, out)
     peaks = load_peaks()
     ms_per_step = max_ms / args.steps
     value = weak_scaling_value(nb_bytes["total"], world, args.steps, max_ms)
@@ -389,6 +401,8 @@ def run_gpu(args, rank, world, local):
             "peak_source": peaks["source"],
             "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
+            # shared-prefix blocks counted once: the bandwidth really needed
+            "frac_unique": round(nb_bytes["unique_total"] / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "traffic": profiled_traffic(sp.name),
             "algorithmic_bytes_per_launch": nb_bytes["total"],
             "us_per_launch": round(dec_ms * 1e3, 3),
@@ -399,6 +413,14 @@ def run_gpu(args, rank, world, local):
             "h2d_bytes_per_step": e2e["h2d"],
             "d2h_bytes_per_step": e2e["d2h"],
             "ms_per_step": round(e2e["ms"] / args.steps, 5),
+            "copies_per_step": e2e["copies_per_step"],
+        },
+        # the host allocator's per-step work (append slots + batch tables) is
+        # not on the device timeline; this adds its measured time to e2e's
+        "e2e_with_alloc": None if e2e is None else {
+            "value": round(nb_bytes["total"] * world / ((e2e["ms"] / args.steps + alloc_us * 1e-3) * 1e-3) / 1e9, 2),
+            "unit": "GB/s",
+            "ms_per_step": round(e2e["ms"] / args.steps + alloc_us * 1e-3, 5),
         },
         "allocator_us_per_step": round(alloc_us, 2),
         "gpu_launches": launches_per_step * args.steps,
@@ -437,26 +459,33 @@ def _build_sequences(alloc, w):
     return seqs, holders
 
 
-def measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out):
+def measure_e2e(args, make_step, stream, q, kn, vn, slots, tables, lens, out):
     """The same step through the C ABI with the per-step inputs in pinned host
-    memory: H2D copies of q, the new K/V, slots, tables and lengths, the
-    kernels, and the D2H copy of the output, all inside the timed region."""
+    memory: q, the new K/V, slots, tables and lengths packed into one pinned
+    staging buffer and sent with one host-to-device copy, the kernels, and one
+    device-to-host copy of the output, all inside the timed region."""
     import torch
 
-    pin = lambda t: t.cpu().pin_memory()
-    h_q, h_kn, h_vn = pin(q), pin(kn), pin(vn)
-    h_slots, h_tables, h_lens = pin(slots), pin(tables), pin(lens)
+    inputs = (q, kn, vn, slots, tables, lens)
+    offs, off = [], 0
+    for t in inputs:
+        off = (off + 255) // 256 * 256           # every input 256-byte aligned in the buffer
+        offs.append(off)
+        off += t.numel() * t.element_size()
+    h_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+    d_buf = torch.empty(off, dtype=torch.uint8, device="cuda")
+    views = []
+    for t, o in zip(inputs, offs):
+        n = t.numel() * t.element_size()
+        h_buf[o:o + n].copy_(t.reshape(-1).view(torch.uint8).cpu())
+        views.append(d_buf[o:o + n].view(t.dtype).view(t.shape))
+    step = make_step(*views)
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_slots, h_tables, h_lens))
+    h2d = sum(t.numel() * t.element_size() for t in inputs)
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
-        q.copy_(h_q, non_blocking=True)
-        kn.copy_(h_kn, non_blocking=True)
-        vn.copy_(h_vn, non_blocking=True)
-        slots.copy_(h_slots, non_blocking=True)
-        tables.copy_(h_tables, non_blocking=True)
-        lens.copy_(h_lens, non_blocking=True)
+        d_buf.copy_(h_buf, non_blocking=True)
         step()
         h_out.copy_(out, non_blocking=True)
 
@@ -472,7 +501,7 @@ def measure_e2e(args, step, stream, q, kn, vn, slots, tables, lens, out):
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1))
     barrier()
-    return dict(ms=e2e_ms, h2d=h2d, d2h=d2h)
+    return dict(ms=e2e_ms, h2d=h2d, d2h=d2h, copies_per_step=2)
 
 
 def allocator_slots(pkv, alloc, w):
@@ -548,10 +577,42 @@ def cpu_baseline(w, nb_bytes, seconds: float) -> dict:
         dt = time.perf_counter() - t0
         if dt >= seconds or reps >= 1000:
             break
-    return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+    value = done / dt / 1e9
+    # the same oracle on one host core, on a smaller sample (about a fifth of
+    # the time budget)
+    one = None
+    if cores > 1:
+        oracle.set_num_threads(1)
+        try:
+            n1 = max(1, int(n * (seconds / 5) / (dt / reps) / cores))
+            s1 = sample[:min(n1, len(sample))]
+            t1 = time.perf_counter()
+            oracle.attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, sp.dtype,
+                             pairs=s1)
+            d1 = time.perf_counter() - t1
+            one = {"value": round(sum(pair_share_bytes(w, int(s)) for s, _ in s1) / d1 / 1e9, 4), "unit": "GB/s",
+                   "cores": 1, "sample": f"{len(s1)} pairs, {d1:.1f} s"}
+        finally:
+            oracle.set_num_threads(cores)
+    return {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"{n} of {len(pairs_all)} (sequence, query head) pairs of {sp.name} x {reps}, fp64 C "
                       f"oracle (gather through block tables + two-pass softmax), {dt:.1f} s",
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), "one_core": one if one is not None else {"value": round(value, 4), "cores": 1}}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or platform.machine()
 
 
 def make_workload(args):
@@ -620,7 +681,7 @@ def run_reference(args, rank, world):
         "data": "synthetic (seeded N(0,1), shapes of the pages' examples)",
         "config": {"workload": sp.name, "description": sp.description, "parallelism": "host CPU"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": sample_desc},
+                         "cpu_model": cpu_model(), "sample": sample_desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -703,26 +764,48 @@ def run_row(args) -> dict:
         out = torch.empty_like(q)
         ws = torch.empty(pkv.pkv_prefill_workspace_bytes(t, hq, hkv, d, mb * bs), dtype=torch.uint8, device="cuda")
         td, qsd, cd = (torch.from_numpy(x).cuda() for x in (tables, qs, ctx))
-        for _ in range(args.warmup):
-            pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
-        t0, t1 = ev(), ev()
-        t0.record()
-        for _ in range(args.steps):
-            pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
-        t1.record()
-        torch.cuda.synchronize()
-        ms = t0.elapsed_time(t1) / args.steps
+
+        def timed(mq: bool) -> float:
+            os.environ["PKV_PREFILL_MQ"] = "1" if mq else "0"
+            try:
+                for _ in range(args.warmup):
+                    pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
+                t0, t1 = ev(), ev()
+                t0.record()
+                for _ in range(args.steps):
+                    pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
+                t1.record()
+                torch.cuda.synchronize()
+            finally:
+                os.environ.pop("PKV_PREFILL_MQ", None)
+            if pkv.pkv_get_last_error() != pkv.PKV_OK:
+                raise RuntimeError("device check failed in the prefill row")
+            return t0.elapsed_time(t1) / args.steps
+
+        ms = timed(True)
+        ms_tok = timed(False)
         # work: each query token attends to its causal window
         windows = np.concatenate([np.arange(c - n + 1, c + 1) for c, n in chunks]).astype(np.int64)
         flops = int(windows.sum()) * hq * d * 2 * 2
         unique = int((ctx.astype(np.int64)).sum()) * hkv * d * 2 * 2
+        peaks = load_peaks()
+        bf16_peak = peaks.get("bf16_tflops", 1590.0)
+        t_hbm = unique / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (bf16_peak * 1e12)
+        bound_s = max(t_hbm, t_tc)
         return {"row": "chunked_prefill", "metric": "chunked prefill + decode step: query tokens/s",
                 "value": round(t / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+                "ms_per_step_per_token_path": round(ms_tok, 4),
+                "speedup_vs_per_token_path": round(ms_tok / ms, 3),
                 "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "unique_kv_gbs": round(unique / (ms * 1e-3) / 1e9, 1),
-                "bf16_peak_tflops": json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"]
-                if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None,
+                "roofline": {"bound": "hbm" if t_hbm >= t_tc else "tensor", "bound_us": round(bound_s * 1e6, 2),
+                             "hbm_us": round(t_hbm * 1e6, 2), "tensor_us": round(t_tc * 1e6, 2),
+                             "frac": round(bound_s / (ms * 1e-3), 4), "hbm_peak_gbs": peaks["hbm_gbs"],
+                             "bf16_peak_tflops": bf16_peak, "peak_source": peaks["source"]},
+                "flops": flops, "unique_kv_bytes": unique,
                 "config": {"shape": "70B GQA 64/8, D128, bs16, bf16", "prefill": "2 x (2048 prefix + 512 chunk)",
-                           "decode": "30 x 4096", "query_tokens": t}}
+                           "decode": "30 x 4096", "query_tokens": t,
+                           "kernels": "multi-query tcgen05 kernel for the chunks, decode kernel for the decode tokens"}}
 
     if args.row == "fp8":
         # the workload's decode over E4M3 pools (1 byte per element + one fp32
@@ -802,6 +885,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass (profiling runs)")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="default workload only (else the 70B, continuous-batching and long-context "
+                         "workloads are measured after it and reported under 'workloads')")
     ap.add_argument("--unfused", action="store_true",
                     help="step = pkv_append + pkv_decode_attention (default: pkv_append_decode_attention)")
     ap.add_argument("--seqs", type=int, default=None,
@@ -816,9 +902,49 @@ def parse_args(argv=None):
     return args
 
 
+# measured after the headline in the default run (same process, same ranks):
+# the two configurations the bandwidth target names and the long-context split
+EXTRA_WORKLOADS = ("llama70b_gqa", "cb_mixed", "long_split")
+
+
+def workload_summary(r: dict) -> dict:
+    """The figures of one extra workload's run kept in the headline line."""
+    keep = {k: r[k] for k in ("value", "unit", "ms_per_step", "tokens_per_s_per_layer",
+                              "algorithmic_bytes_per_step", "unique_bytes_per_step", "dtype", "clocks")}
+    keep["config"] = {k: r["config"][k] for k in ("workload", "description", "partition", "step_call")}
+    keep["roofline"] = {k: r["roofline"][k] for k in ("kernel", "achieved", "peak", "unit", "frac", "frac_unique",
+                                                      "traffic", "us_per_launch")}
+    if r.get("e2e"):
+        keep["e2e"] = {k: r["e2e"][k] for k in ("value", "unit", "ms_per_step")}
+    return keep
+
+
+def relaunch_per_gpu(argv, n: int) -> int:
+    """Run this script once per GPU (torch.distributed.run, one node,
+    rendezvous on 127.0.0.1) and return the launcher's exit status."""
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=3600)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, 9)
+        proc.wait()
+        return 124
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     args = parse_args(argv)
     rank, world, local = dist_env()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not args.row:
+        # `bench.py --gpus N` outside a launcher: one process per GPU
+        return relaunch_per_gpu(argv, args.gpus)
     if args.row:
         if rank == 0:
             print(json.dumps(run_row(args)), flush=True)
@@ -837,6 +963,21 @@ def main(argv=None):
                                 device_id=torch.device("cuda", local))
     try:
         result = run_gpu(args, rank, world, local)
+        if not args.no_extra_workloads and args.workload == DEFAULT_WORKLOAD and args.seqs is None:
+            import copy
+
+            import torch
+            import workloads
+
+            subs = {}
+            for name in EXTRA_WORKLOADS:
+                a2 = copy.copy(args)
+                a2.workload = name
+                a2.partition = workloads.CONFIGS[name].partition_tokens or 0
+                a2.no_cpu_baseline = True
+                subs[name] = workload_summary(run_gpu(a2, rank, world, local))
+                torch.cuda.empty_cache()
+            result["workloads"] = subs
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:

@@ -55,3 +55,23 @@ def test_two_rank_timing_reduction_and_weak_scaling():
         assert slowest == 15.0                          # max over ranks
         assert value == pytest.approx(2 * 4 * 1.0 / 15e-3)  # 2 ranks x 4 steps x 1 GB / 15 ms
     assert got[1][3] == 0
+
+
+def test_gpus_flag_launches_one_process_per_rank():
+    # `bench.py --gpus 2` outside a launcher starts two ranks itself; the
+    # reference arm (host only) runs on rank 0 and reports both ranks
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    env.pop("WORLD_SIZE", None)
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "3", "--warmup", "3"], capture_output=True, text=True,
+                       timeout=600, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
