@@ -242,7 +242,10 @@ def run_gpu(args, rank, world, local):
     # returning them to the LIFO free list in reverse, then every sequence is
     # built up to ctx - 1 tokens (prefix blocks shared through fork).
     alloc = pkv.BlockAllocator(w.num_blocks, sp.block_size)
-    slots_np, alloc_us = allocator_slots(pkv, alloc, w)
+    slots_np, alloc_us, groups = allocator_slots(pkv, alloc, w)
+    # a workload whose sequences share prefix blocks runs its step through the
+    # shared-prefix call (each group's prefix read once); --no-cascade: plain
+    cascade = groups is not None and not args.no_cascade and not args.unfused
 
     q = dev(w.q)
     kc, vc = dev(w.k_cache), dev(w.v_cache)
@@ -260,6 +263,15 @@ def run_gpu(args, rank, world, local):
     merge_launched = part != pkv.PKV_PARTITION_NONE and not (
         part > 0 and -(-w.max_blocks_per_seq * sp.block_size // part) <= 1)
     launches_per_step = (1 if not args.unfused else 2) + (1 if merge_launched else 0)
+    if cascade:
+        starts_np, claims_np = groups
+        gstart = torch.from_numpy(starts_np).cuda()
+        claims = torch.from_numpy(claims_np).cuda()
+        ngroups = len(starts_np) - 1
+        n = pkv.pkv_shared_prefix_workspace_bytes(sp.num_seqs, sp.num_q_heads, sp.num_kv_heads, sp.head_dim,
+                                                  w.max_blocks_per_seq * sp.block_size, ngroups)
+        ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+        launches_per_step = 4  # preparation, shared-prefix kernel, decode kernel, merge
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if args.flush_l2 else None
 
@@ -277,13 +289,23 @@ def run_gpu(args, rank, world, local):
     c_append, c_decode = pkv.lib.pkv_append, pkv.lib.pkv_decode_attention
     c_fused = pkv.lib.pkv_append_decode_attention
     fused_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr()) + decode_args
+    if cascade:
+        # the step's one call: append + shared-prefix decode
+        c_fused = pkv.lib.pkv_append_decode_attention_shared_prefix
+        fused_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr(), q.data_ptr(), q.shape[0], q.shape[1], kdesc,
+                      vdesc, tables.data_ptr(), tables.shape[1], lens.data_ptr(), gstart.data_ptr(), ngroups,
+                      claims.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, sptr)
 
-    def make_step(q, kn, vn, slots, tables, lens):
+    def make_step(q, kn, vn, slots, tables, lens, gstart=None, claims=None):
         """The step's raw C ABI calls on these device inputs."""
         a_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr(), slots.numel(), kdesc, vdesc, sptr)
         d_args = (q.data_ptr(), q.shape[0], q.shape[1], kdesc, vdesc, tables.data_ptr(), tables.shape[1],
                   lens.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, part, sptr)
         f_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr()) + d_args
+        if cascade:
+            f_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr(), q.data_ptr(), q.shape[0], q.shape[1], kdesc,
+                      vdesc, tables.data_ptr(), tables.shape[1], lens.data_ptr(), gstart.data_ptr(), ngroups,
+                      claims.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, sptr)
         if args.unfused:
             def step():
                 c_append(*a_args)
@@ -293,12 +315,17 @@ def run_gpu(args, rank, world, local):
                 c_fused(*f_args)
         return step
 
-    step = make_step(q, kn, vn, slots, tables, lens)
+    step_inputs = (q, kn, vn, slots, tables, lens) + ((gstart, claims) if cascade else ())
+    step = make_step(*step_inputs)
 
     # the binding path once, with its argument checks
     pkv.pkv_append(kn, vn, slots, kc, vc, stream)
     pkv.pkv_decode_attention(q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
-    pkv.pkv_append_decode_attention(kn, vn, slots, q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
+    if cascade:
+        pkv.pkv_append_decode_attention_shared_prefix(kn, vn, slots, q, kc, vc, tables, lens, gstart, claims,
+                                                      w.scale, out, ws, stream)
+    else:
+        pkv.pkv_append_decode_attention(kn, vn, slots, q, kc, vc, tables, lens, w.scale, out, ws, part, stream)
     with nvtx("pkv warm-up"):
         for _ in range(args.warmup):
             step()
@@ -353,7 +380,7 @@ def run_gpu(args, rank, world, local):
 
     # ---- end to end through the C ABI with host buffers
     with nvtx("pkv end-to-end"):
-        e2e = None if args.no_e2e else measure_e2e(args, make_step, stream, q, kn, vn, slots, tables, lens, out)
+        e2e = None if args.no_e2e else measure_e2e(args, make_step, stream, step_inputs, out)
     peaks = load_peaks()
     ms_per_step = max_ms / args.steps
     value = weak_scaling_value(nb_bytes["total"], world, args.steps, max_ms)
@@ -386,7 +413,8 @@ def run_gpu(args, rank, world, local):
             "products": "ffma (CUDA-core variant)" if os.environ.get("PKV_FMA") == "1" else "mma m16n8k16",
             "l2": "flushed between steps" if args.flush_l2 else "per-step KV working set > L2 (no flush)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "step_call": "pkv_append + pkv_decode_attention" if args.unfused else "pkv_append_decode_attention",
+            "step_call": ("pkv_append + pkv_decode_attention" if args.unfused else
+                          "pkv_append_decode_attention_shared_prefix" if cascade else "pkv_append_decode_attention"),
         },
         "tokens_per_s_per_layer": round(sp.num_seqs * world / (ms_per_step * 1e-3), 1),
         "algorithmic_bytes_per_step": nb_bytes["total"],
@@ -395,7 +423,8 @@ def run_gpu(args, rank, world, local):
         "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
         "roofline": {
             "bound": "hbm",
-            "kernel": "paged_decode_kernel" + ("+lse_merge_kernel" if merge_launched else ""),
+            "kernel": ("cascade_prep_kernel+mq_attention_kernel+" if cascade else "") + "paged_decode_kernel" +
+                      ("+lse_merge_kernel" if merge_launched else ""),
             "achieved": round(achieved, 2),
             "peak": peaks["hbm_gbs"],
             "peak_source": peaks["source"],
@@ -459,14 +488,14 @@ def _build_sequences(alloc, w):
     return seqs, holders
 
 
-def measure_e2e(args, make_step, stream, q, kn, vn, slots, tables, lens, out):
+def measure_e2e(args, make_step, stream, inputs, out):
     """The same step through the C ABI with the per-step inputs in pinned host
-    memory: q, the new K/V, slots, tables and lengths packed into one pinned
-    staging buffer and sent with one host-to-device copy, the kernels, and one
-    device-to-host copy of the output, all inside the timed region."""
+    memory: q, the new K/V, slots, tables and lengths (and the sharing groups,
+    when the step uses them) packed into one pinned staging buffer and sent
+    with one host-to-device copy, the kernels, and one device-to-host copy of
+    the output, all inside the timed region."""
     import torch
 
-    inputs = (q, kn, vn, slots, tables, lens)
     offs, off = [], 0
     for t in inputs:
         off = (off + 255) // 256 * 256           # every input 256-byte aligned in the buffer
@@ -532,10 +561,11 @@ def allocator_slots(pkv, alloc, w):
     t0 = time.perf_counter()
     slots = alloc.append_slots(seqs)
     tables, lens = alloc.batch_tables(seqs, w.max_blocks_per_seq)
+    groups = alloc.prefix_groups(seqs) if w.spec.share_group else None
     alloc_us = (time.perf_counter() - t0) * 1e6
     if not (np.array_equal(tables, w.block_tables) and np.array_equal(lens, w.context_lens)):
         raise RuntimeError("allocator tables differ from the workload's")
-    return slots, alloc_us
+    return slots, alloc_us, groups
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
@@ -765,15 +795,19 @@ def run_row(args) -> dict:
         ws = torch.empty(pkv.pkv_prefill_workspace_bytes(t, hq, hkv, d, mb * bs), dtype=torch.uint8, device="cuda")
         td, qsd, cd = (torch.from_numpy(x).cuda() for x in (tables, qs, ctx))
 
-        def timed(mq: bool) -> float:
+        def timed(mq: bool, nseq: int = len(chunks)) -> float:
+            # nseq < len(chunks): the first nseq sequences only (the chunks)
             os.environ["PKV_PREFILL_MQ"] = "1" if mq else "0"
+            tt = int(qs[nseq])
+            qq, oo = q[:tt], out[:tt]
+            tq, qq_s, cc = td[:nseq], qsd[:nseq + 1], cd[:nseq]
             try:
                 for _ in range(args.warmup):
-                    pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
+                    pkv.pkv_prefill_attention(qq, kc, vc, tq, qq_s, cc, 0.088, oo, ws)
                 t0, t1 = ev(), ev()
                 t0.record()
                 for _ in range(args.steps):
-                    pkv.pkv_prefill_attention(q, kc, vc, td, qsd, cd, 0.088, out, ws)
+                    pkv.pkv_prefill_attention(qq, kc, vc, tq, qq_s, cc, 0.088, oo, ws)
                 t1.record()
                 torch.cuda.synchronize()
             finally:
@@ -782,11 +816,18 @@ def run_row(args) -> dict:
                 raise RuntimeError("device check failed in the prefill row")
             return t0.elapsed_time(t1) / args.steps
 
+        if args.chunks_only:
+            # profiling case: the two prefill chunks alone, multi-query kernel only
+            ms_chunks = timed(True, 2)
+            return {"row": "chunked_prefill_chunks_only", "ms_per_step": round(ms_chunks, 4),
+                    "steps": args.steps, "warmup": args.warmup}
         ms = timed(True)
         ms_tok = timed(False)
+        ms_chunks = timed(True, 2)     # the two prefill chunks alone (multi-query kernel)
         # work: each query token attends to its causal window
         windows = np.concatenate([np.arange(c - n + 1, c + 1) for c, n in chunks]).astype(np.int64)
         flops = int(windows.sum()) * hq * d * 2 * 2
+        flops_chunks = int(windows[:int(qs[2])].sum()) * hq * d * 2 * 2
         unique = int((ctx.astype(np.int64)).sum()) * hkv * d * 2 * 2
         peaks = load_peaks()
         bf16_peak = peaks.get("bf16_tflops", 1590.0)
@@ -796,6 +837,8 @@ def run_row(args) -> dict:
         return {"row": "chunked_prefill", "metric": "chunked prefill + decode step: query tokens/s",
                 "value": round(t / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
                 "ms_per_step_per_token_path": round(ms_tok, 4),
+                "ms_chunks_only": round(ms_chunks, 4),
+                "chunks_only_tflops": round(flops_chunks / (ms_chunks * 1e-3) / 1e12, 2),
                 "speedup_vs_per_token_path": round(ms_tok / ms, 3),
                 "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "unique_kv_gbs": round(unique / (ms * 1e-3) / 1e9, 1),
                 "roofline": {"bound": "hbm" if t_hbm >= t_tc else "tensor", "bound_us": round(bound_s * 1e6, 2),
@@ -890,6 +933,10 @@ def parse_args(argv=None):
                          "workloads are measured after it and reported under 'workloads')")
     ap.add_argument("--unfused", action="store_true",
                     help="step = pkv_append + pkv_decode_attention (default: pkv_append_decode_attention)")
+    ap.add_argument("--chunks-only", action="store_true",
+                    help="--row prefill: time only the two prefill chunks (a small case for profiling)")
+    ap.add_argument("--no-cascade", action="store_true",
+                    help="workloads with shared prefixes: plain decode step instead of the shared-prefix call")
     ap.add_argument("--seqs", type=int, default=None,
                     help="run the workload with its first N sequences only (small profiling cases)")
     args = ap.parse_args(argv)

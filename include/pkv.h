@@ -242,11 +242,16 @@ pkv_status pkv_append_decode_attention(const void *k_new, const void *v_new,
  *
  * Query i of sequence s attends causally to positions 0 .. ctx_s - n_s + i.
  * A decode sequence is a chunk of one, so prefill chunks and decode tokens
- * go in one call.  Each query token runs as its own decode over its causal
- * prefix (sharing the sequence's table row), on the decode kernel; the
- * chunk's tokens re-read the shared prefix, mostly from L2.  Inconsistent
- * lengths (n_s < 1, ctx_s < n_s) are flagged on the device and give zero
- * rows.  Same limits as pkv_decode_attention; T < 2^24.
+ * go in one call.  Chunks of two or more tokens run on a multi-query
+ * tensor-core kernel (tcgen05, fp32 accumulators in tensor memory): blocks
+ * of 128 / G tokens x the G query heads of one KV head form 128-row tiles
+ * that read each K/V tile of their causal range once.  Decode tokens run on
+ * the decode kernel.  (Environment PKV_PREFILL_MQ=0 sends every token
+ * through the decode kernel instead -- the path before the multi-query
+ * kernel, kept for comparison.)  Inconsistent lengths (n_s < 1, ctx_s < n_s)
+ * are flagged on the device and give zero rows.  Same limits as
+ * pkv_decode_attention; T < 2^24; the multi-query kernel needs G <= 128,
+ * B <= 4096 and scale != 0 (otherwise every token takes the decode kernel).
  * ------------------------------------------------------------------------ */
 pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_seqs, int64_t num_q_heads,
                                  pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
@@ -255,6 +260,52 @@ pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_
                                  size_t workspace_bytes, pkv_stream stream);
 size_t pkv_prefill_workspace_bytes(int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
                                    int64_t head_dim, int64_t max_context_len);
+
+/* --------------------------------------------------------------------------
+ * pkv_append_decode_attention_shared_prefix -- a decode step (with an
+ * optional fused append) for a batch in which groups of sequences share the
+ * blocks of a common prefix.  [KVB] "Prefix caching": many requests share a
+ * prefix (a system prompt, few-shot examples); [ENG] "The Elegant Fix":
+ * requests with the same prompt prefix share pages instead of duplicating
+ * them.  The result is exactly pkv_append_decode_attention's (attention over
+ * each sequence's whole context); only the way it is computed differs: each
+ * shared prefix is read once per group and scored against every member's
+ * query heads together on the tensor cores (M = members x G rows), each
+ * sequence's own blocks after it go through the decode kernel, which resumes
+ * from the prefix's fp32 partial (max, sum, weighted V) -- no extra merge.
+ *
+ *   k_new, v_new, slot_mapping   as for pkv_append_decode_attention, or all
+ *                  three NULL for no append
+ *   group_start    device int32 [num_groups + 1]: group g is sequences
+ *                  group_start[g] .. group_start[g+1]-1 (consecutive in the
+ *                  batch); group_start[0] = 0, group_start[num_groups] = B,
+ *                  non-decreasing.  A sequence sharing nothing is a group
+ *                  of one.
+ *   shared_lens    device int32 [B]: claimed number of leading positions of
+ *                  each sequence stored in blocks shared with its group
+ *                  (e.g. from pkv_batch_prefix_groups)
+ *   workspace      >= pkv_shared_prefix_workspace_bytes(...)
+ *
+ * The kernel takes as the group's reference the first member with the
+ * largest claim, and uses for each member only whole blocks that (a) are
+ * within its claim, (b) end before its last position (the position of this
+ * step's new token stays in the sequence's own block) and (c) have the same
+ * table entries as the reference's: a wrong claim only shrinks the shared
+ * part, never changes the result.  An invalid group_start entry is flagged
+ * (PKV_ERR_DEVICE_CHECK) and that group computed without sharing.
+ * Limits: those of pkv_decode_attention, 16-bit pools, G <= 128,
+ * num_groups <= 4096; num_groups == 0 (or scale == 0) runs the plain step.
+ * ------------------------------------------------------------------------ */
+pkv_status pkv_append_decode_attention_shared_prefix(
+    const void *k_new, const void *v_new, const int64_t *slot_mapping, const void *q, int64_t num_seqs,
+    int64_t num_q_heads, pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+    int64_t max_blocks_per_seq, const int32_t *context_lens, const int32_t *group_start, int64_t num_groups,
+    const int32_t *shared_lens, float scale, void *out, void *workspace, size_t workspace_bytes,
+    pkv_stream stream);
+/* Bytes of workspace for pkv_append_decode_attention_shared_prefix on the
+ * current device (0 for invalid arguments). */
+size_t pkv_shared_prefix_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                         int64_t head_dim, int64_t max_context_len, int64_t num_groups);
 
 /* --------------------------------------------------------------------------
  * pkv_decode_attention_static_scratch -- pkv_decode_attention for callers
@@ -376,6 +427,16 @@ int64_t pkv_seq_context_len(void *h, int32_t seq);
 pkv_status pkv_batch_tables(void *h, const int32_t *seqs, int32_t n, int32_t *dst,
                             int32_t cap, int32_t *context_lens);
 
+/* Sharing groups of a batch (host), for
+ * pkv_append_decode_attention_shared_prefix: consecutive sequences of
+ * seqs[0..n) whose first block is one and the same shared block (refcount >
+ * 1) form a group, any other sequence a group of its own.  group_start[0 ..
+ * *num_groups] receives the groups (capacity n + 1), shared_lens[i] the
+ * number of leading positions of seqs[i] held in shared blocks (its leading
+ * blocks with refcount > 1, times bs). */
+pkv_status pkv_batch_prefix_groups(void *h, const int32_t *seqs, int32_t n, int32_t *group_start,
+                                   int32_t *num_groups, int32_t *shared_lens);
+
 /* Testing hook for the kernels' bounded waits (no counterpart on the pages).
  * With enable != 0, decode launches made afterwards by this process issue no
  * tile copies, so every wait for a tile runs out after wait_limit_ns (clamped
@@ -384,6 +445,12 @@ pkv_status pkv_batch_tables(void *h, const int32_t *seqs, int32_t n, int32_t *ds
  * enable == 0 restores normal operation (2 s limit).  Host-side setting only;
  * nothing faults, traps or hangs. */
 pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns);
+
+/* Testing hook (no counterpart on the pages): y[i] = 2^x[i] computed the way
+ * the multi-query kernel computes part of its softmax exponentials on the
+ * FMA pipes (PKV_MQ_POLY=1): round-to-nearest range reduction and a degree-4
+ * polynomial, relative error < 1e-5; 0 below -126.  x, y: device float [n]. */
+pkv_status pkv_test_exp2_poly(const float *x, float *y, int64_t n, pkv_stream stream);
 
 /* Text of the last CUDA runtime error a call of this thread reported as
  * PKV_ERR_CUDA ("no error" if none); static storage. */

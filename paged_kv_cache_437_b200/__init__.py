@@ -114,6 +114,13 @@ def _load():
         "pkv_decode_attention_static_scratch": (ctypes.c_int, [_c_vp, _c_i64, _c_i64, pkv_cache, pkv_cache,
                                                                _c_vp, _c_i64, _c_vp, ctypes.c_float, _c_vp,
                                                                _c_i32, _c_vp]),
+        "pkv_append_decode_attention_shared_prefix": (ctypes.c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
+                                                                     pkv_cache, pkv_cache, _c_vp, _c_i64, _c_vp,
+                                                                     _c_vp, _c_i64, _c_vp, ctypes.c_float, _c_vp,
+                                                                     _c_vp, _c_sz, _c_vp]),
+        "pkv_shared_prefix_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64]),
+        "pkv_batch_prefix_groups": (ctypes.c_int, [_c_vp, _c_vp, _c_i32, _c_vp, ctypes.POINTER(_c_i32), _c_vp]),
+        "pkv_test_exp2_poly": (ctypes.c_int, [_c_vp, _c_vp, _c_i64, _c_vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -472,6 +479,59 @@ def pkv_batch_tables(h, seqs, cap: int):
     return tables, lens
 
 
+def pkv_batch_prefix_groups(h, seqs):
+    """(group_start [G+1] int32, shared_lens [n] int32) of a batch: runs of
+    consecutive sequences that start with the same shared block."""
+    import numpy as np
+
+    s = np.ascontiguousarray(seqs, dtype=np.int32)
+    starts = np.empty(len(s) + 1, dtype=np.int32)
+    shared = np.empty(len(s), dtype=np.int32)
+    ng = _c_i32(0)
+    _check(lib.pkv_batch_prefix_groups(h, s.ctypes.data, len(s), starts.ctypes.data, ctypes.byref(ng),
+                                       shared.ctypes.data), "pkv_batch_prefix_groups")
+    return starts[:ng.value + 1].copy(), shared
+
+
+def pkv_shared_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                      max_context_len: int, num_groups: int) -> int:
+    return int(lib.pkv_shared_prefix_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                     max_context_len, num_groups))
+
+
+def pkv_append_decode_attention_shared_prefix(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables,
+                                              context_lens, group_start, shared_lens, scale: float, out,
+                                              workspace, stream=None) -> None:
+    """A decode step (append optional: k_new = v_new = slot_mapping = None)
+    whose sharing groups' common prefixes are read once per group."""
+    import torch
+
+    _check_decode_args(q, k_cache, block_tables, context_lens, out)
+    for t, n in ((group_start, "group_start"), (shared_lens, "shared_lens"), (workspace, "workspace")):
+        _require(t, n)
+    if group_start.dtype != torch.int32 or shared_lens.dtype != torch.int32:
+        raise TypeError("group_start and shared_lens must be int32")
+    b = q.shape[0]
+    if shared_lens.numel() != b or group_start.numel() < 1:
+        raise ValueError("shapes: group_start [G+1], shared_lens [B]")
+    ptrs = (None, None, None)
+    if k_new is not None or v_new is not None or slot_mapping is not None:
+        for t, n in ((k_new, "k_new"), (v_new, "v_new"), (slot_mapping, "slot_mapping")):
+            _require(t, n)
+        if slot_mapping.dtype != torch.int64 or k_new.dtype != q.dtype or v_new.dtype != q.dtype:
+            raise TypeError("slot_mapping int64; k_new / v_new in q's dtype")
+        if k_new.shape != (b, k_cache.shape[1], k_cache.shape[3]) or v_new.shape != k_new.shape or \
+                slot_mapping.numel() != b:
+            raise ValueError("shapes: k_new/v_new [B][Hkv][D], slot_mapping [B]")
+        ptrs = (k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr())
+    st = lib.pkv_append_decode_attention_shared_prefix(
+        *ptrs, q.data_ptr(), b, q.shape[1], cache_desc(k_cache), cache_desc(v_cache), block_tables.data_ptr(),
+        block_tables.shape[1], context_lens.data_ptr(), group_start.data_ptr(), group_start.numel() - 1,
+        shared_lens.data_ptr(), float(scale), out.data_ptr(), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(st, "pkv_append_decode_attention_shared_prefix")
+
+
 class BlockAllocator:
     """Owning wrapper of one allocator handle."""
 
@@ -506,6 +566,7 @@ class BlockAllocator:
     block_table = lambda self, s: pkv_seq_block_table(self.handle, s)
     context_len = lambda self, s: pkv_seq_context_len(self.handle, s)
     batch_tables = lambda self, seqs, cap: pkv_batch_tables(self.handle, seqs, cap)
+    prefix_groups = lambda self, seqs: pkv_batch_prefix_groups(self.handle, seqs)
 
 
 class Scheduler:

@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpkv.so")
 SOURCES = [os.path.join(CSRC, "pkv_cuda.cu"), os.path.join(CSRC, "allocator.cpp"),
            os.path.join(CSRC, "scheduler.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("decode.cuh", "ptx.cuh")] + [os.path.join(INCLUDE, "pkv.h")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("decode.cuh", "mq_attention.cuh", "ptx.cuh")] + [os.path.join(INCLUDE, "pkv.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

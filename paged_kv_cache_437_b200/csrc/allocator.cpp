@@ -346,6 +346,34 @@ pkv_status pkv_batch_tables(void *h, const int32_t *seqs, int32_t n, int32_t *ds
     return PKV_OK;
 }
 
+pkv_status pkv_batch_prefix_groups(void *h, const int32_t *seqs, int32_t n, int32_t *group_start,
+                                   int32_t *num_groups, int32_t *shared_lens) {
+    Allocator *a = as_alloc(h);
+    if (!a || n < 0 || !group_start || !num_groups || (n > 0 && (!seqs || !shared_lens)))
+        return PKV_ERR_INVALID;
+    for (int32_t i = 0; i < n; ++i)
+        if (!a->valid_seq(seqs[i]))
+            return PKV_ERR_INVALID;
+    int32_t ng = 0;
+    int32_t group_first = -1;  // first block shared by the open group, -1: none
+    for (int32_t i = 0; i < n; ++i) {
+        const Sequence &q = a->seqs[seqs[i]];
+        const int32_t first = q.blocks.empty() ? -1 : q.blocks[0];
+        const bool shared_first = first >= 0 && a->refcount[first] > 1;
+        if (i == 0 || !shared_first || first != group_first) {
+            group_start[ng++] = i;
+            group_first = shared_first ? first : -1;
+        }
+        size_t k = 0;
+        while (k < q.blocks.size() && a->refcount[q.blocks[k]] > 1)
+            ++k;
+        shared_lens[i] = (int32_t)(k * (size_t)a->block_size);
+    }
+    group_start[ng] = n;
+    *num_groups = ng;
+    return PKV_OK;
+}
+
 const char *pkv_status_string(pkv_status s) {
     switch (s) {
     case PKV_OK: return "ok";

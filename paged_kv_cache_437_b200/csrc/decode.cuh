@@ -88,6 +88,13 @@ struct DecodeArgs {
     // chunked prefill: "sequence" s reads block-table row table_rows[s]
     // (several query tokens of one sequence share its row); null = row s
     const int32_t *table_rows;
+    // shared-prefix cascade (16-bit MMA path): sequence s starts
+    // table_offset[s] entries into its table row (its positions before that
+    // were attended by the shared-prefix kernel), and a unit that starts a
+    // row with table_offset[s] > 0 resumes from that kernel's fp32 partial
+    // (init_o [B][Hq][D] relative to 2^init_m, init_l; log2 domain); null = none
+    const int32_t *table_offset;
+    const float *init_o, *init_m, *init_l;
 };
 
 struct SmemLayout {
@@ -164,6 +171,7 @@ __device__ __forceinline__ int upper_bound_i(const int *a, int n, long long x) {
 struct Seg {
     int seq, pair, t0, t1, ctx, dest;  // dest < 0: final output, else partial index
     int trow;                          // block-table row of the sequence
+    int toff;                          // entries of that row to skip
 };
 
 struct Walker {
@@ -203,8 +211,10 @@ __device__ __forceinline__ bool walker_next_raw(Walker &w, Seg &sg, const Decode
 __device__ __forceinline__ bool walker_next(Walker &w, Seg &sg, const DecodeArgs &a,
                                             const int *prefix, const int *ctxs, int gw) {
     const bool has = walker_next_raw(w, sg, a, prefix, ctxs, gw);
-    if (has)
+    if (has) {
         sg.trow = a.table_rows ? __ldg(a.table_rows + sg.seq) : sg.seq;
+        sg.toff = a.table_offset ? __ldg(a.table_offset + sg.seq) : 0;
+    }
     return has;
 }
 
@@ -407,6 +417,18 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         for (int s = blockIdx.x; s < a.B; s += gridDim.x) {
             if (ctxs[s] != 0)
                 continue;
+            if (!FP8 && !FMA && a.init_l && a.table_offset && __ldg(a.table_offset + s) > 0) {
+                // nothing after the shared prefix: its partial, normalized
+                uint32_t *o = reinterpret_cast<uint32_t *>(a.out + (size_t)s * a.Hq * D);
+                for (int i = threadIdx.x; i < a.Hq * D / 2; i += blockDim.x) {
+                    const size_t row = (size_t)s * a.Hq + (2 * i) / D;
+                    const float l = __ldg(a.init_l + row);
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    const float2 v = __ldg(reinterpret_cast<const float2 *>(a.init_o + row * D) + (i % (D / 2)));
+                    o[i] = pack2<BF16>(v.x * inv, v.y * inv);
+                }
+                continue;
+            }
             uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)s * a.Hq * D);
             const int n = a.Hq * D / 8;
             for (int i = threadIdx.x; i < n; i += blockDim.x)
@@ -469,7 +491,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const int nblk = ceil_div_i(ns.ctx, a.bs);
             nx_seq = ns.seq;
             nx_base = lb;
-            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.trow * a.mb + lb + lane) : 0;
+            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.trow * a.mb + ns.toff + lb + lane) : 0;
         }
     };
     // set when the producer enters a unit; the prefetch for the unit after it
@@ -488,7 +510,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 nx_seq = -1;
             } else {
                 const int nblk = ceil_div_i(ps.ctx, a.bs);
-                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.trow * a.mb + lb + lane) : 0;
+                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.trow * a.mb + ps.toff + lb + lane) : 0;
             }
         }
         if (want_prefetch) {
@@ -661,6 +683,33 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
             m_run[nt][0] = m_run[nt][1] = -INFINITY;
             l_run[nt][0] = l_run[nt][1] = 0.f;
+        }
+
+        if constexpr (!FP8 && !FMA) {
+            if (a.init_l != nullptr && cs.t0 == 0 && cs.toff > 0) {
+                // the row's positions before its own blocks were attended by
+                // the shared-prefix kernel: resume from its partial.  Lane
+                // (g8, c4) holds heads 2c4, 2c4+1 of each n-tile at d = 16 mt +
+                // g8 (+8); the sum l is kept once per head (lane g8 == 0).
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int head = nt * 8 + 2 * c4 + j;
+                        if (head < rows) {
+                            const size_t row = (size_t)cs.seq * a.Hq + h0 + head;
+                            m_run[nt][j] = __ldg(a.init_m + row);
+                            l_run[nt][j] = g8 == 0 ? __ldg(a.init_l + row) : 0.f;
+                            const float *po = a.init_o + row * D;
+#pragma unroll
+                            for (int mt = 0; mt < kMT; ++mt) {
+                                o[nt][mt][j] = __ldg(po + 16 * mt + g8);
+                                o[nt][mt][2 + j] = __ldg(po + 16 * mt + g8 + 8);
+                            }
+                        }
+                    }
+                }
+            }
         }
 
         for (int t = cs.t0; t < cs.t1; ++t) {
@@ -1625,7 +1674,14 @@ __global__ void __launch_bounds__(256) prefill_expand_kernel(const int32_t *__re
                                                              const int32_t *__restrict__ context_lens,
                                                              int B, int T, int64_t cap,
                                                              int32_t *__restrict__ lens,
-                                                             int32_t *__restrict__ rows, unsigned *err) {
+                                                             int32_t *__restrict__ rows, int *mq_counter,
+                                                             unsigned *err) {
+    // with the multi-query kernel enabled (mq_counter != null), chunks of two
+    // or more tokens are its work: their tokens get length 0 here (a zero
+    // row from the decode kernel, overwritten by the multi-query kernel,
+    // which runs after it in the stream) and its unit counter starts at 0
+    if (mq_counter && blockIdx.x == 0 && threadIdx.x == 0)
+        *mq_counter = 0;
     for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < T; j += gridDim.x * blockDim.x) {
         int lo = 0, hi = B + 1;  // first index with query_start > j
         while (lo < hi) {
@@ -1642,6 +1698,8 @@ __global__ void __launch_bounds__(256) prefill_expand_kernel(const int32_t *__re
         int len = c - n + (j - q0) + 1;
         if (n <= 0 || c < n || c > cap || j < q0 || j >= q0 + n) {
             atomicOr(err, kErrContext);
+            len = 0;
+        } else if (mq_counter && n >= 2) {
             len = 0;
         }
         lens[j] = len;

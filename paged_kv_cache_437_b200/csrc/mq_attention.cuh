@@ -1,0 +1,760 @@
+// Multi-query paged attention on the 5th-generation tensor cores (tcgen05).
+//
+// What is computed ("LLM Inference: KV Cache, Batching & Scheduling",
+// cariara.com, section "Chunked prefill": a prompt is fed in fixed-size
+// chunks, e.g. 512 tokens, interleaved with other requests' decode steps):
+// query i (0-based) of a chunk of n tokens whose sequence has context c after
+// the chunk's append attends, for every query head, to positions
+// 0 .. c - n + i of that sequence's paged cache -- causal inside the chunk,
+// everything before it.
+//
+// Kernel design (B200):
+//  * Work unit = (sequence, KV head, block of `tpb` consecutive chunk tokens).
+//    Its rows are the tpb tokens x the G query heads that share the KV head
+//    (tpb * G <= 128): one 128-row tile.  Every K/V tile of the unit's
+//    causal range is loaded once for all of them, so a chunk reads each K/V
+//    position once per row block instead of once per query token.
+//  * S = Q K^T and O += P V are tcgen05.mma (kind::f16, M = 128) with both
+//    operands in shared memory (128-byte swizzled tiles straight from TMA)
+//    and fp32 accumulators in tensor memory: S double-buffered (2 x 128
+//    columns), O in 128 columns.
+//  * Warp roles in a 192-thread CTA: warps 0-3 own one row each (TMEM lane =
+//    row): online softmax of S, P to shared memory, the rare O rescale and
+//    the epilogue; warp 4 is the producer (unit scheduler, TMA loads of Q and
+//    of the K/V tiles through the block table); warp 5 allocates TMEM and one
+//    of its threads issues every MMA.  All hand-offs are mbarriers; every
+//    wait is bounded (time-out -> error word, orderly teardown).
+//  * Persistent grid (one CTA per SM); units are taken from a global counter
+//    in order of decreasing causal length within each sequence.
+//  * Online softmax in the log2 domain with a lazy rescale: the running
+//    reference max only moves when the tile max exceeds it by more than 2^8,
+//    so P stays <= 256 (exact enough in 16 bits) and O in TMEM is almost
+//    never rescaled.  Positions past a row's causal limit get -inf before the
+//    exponential; V rows past the context are zeroed in shared memory before
+//    the P V product (0 * NaN would otherwise leak a poisoned slot).
+#pragma once
+
+#include "decode.cuh"
+
+namespace pkv {
+
+constexpr int kMqRows = 128;      // MMA M: query rows of one unit
+constexpr int kMqTile = 128;      // KV positions per tile (N of Q K^T, K of P V)
+constexpr int kMqThreads = 192;   // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr int kMqKStages = 2;     // K tiles in flight
+constexpr int kMqVStages = 2;     // V tiles in flight
+constexpr float kMqRescaleLog2 = 8.0f;
+constexpr int kMqMaxSeqs = 4096;  // per-sequence unit prefix kept in shared memory
+
+enum MqMode : int {
+    kMqPrefill = 0,  // chunks of query tokens, causal limits, normalized output
+    kMqPrefix = 1,   // decode queries of a sharing group over its common prefix, fp32 partials
+};
+
+struct MqArgs {
+    int mode;
+    uint16_t *out;                 // prefill: [T][Hq][D]
+    const int32_t *block_tables;   // [B][MB]
+    const int32_t *query_start;    // prefill: [B + 1]
+    const int32_t *context_lens;   // prefill: [B], after the chunk's append
+    // shared-prefix groups: members of group g are sequences
+    // group_start[g] .. group_start[g+1]-1; the group's common blocks are read
+    // through row group_ref[g] of the table, up to position group_len[g];
+    // member s attends to its first shared[s] positions there
+    const int32_t *group_start, *group_ref, *group_len, *shared;
+    float *part_o, *part_m, *part_l;  // prefix: [B][Hq][D], [B][Hq], [B][Hq] (log2-domain max)
+    int nsrc;                      // sources of units: sequences (prefill) or groups (prefix)
+    int64_t mb;                    // MB
+    int64_t nb;                    // NB
+    int B, T, Hq, Hkv, G, bs, tpb;
+    float scale_log2;              // |scale| * log2(e)
+    int negate_q;                  // scale < 0: the score product negates Q
+    int *unit_counter;             // zero at launch (written by the expansion kernel)
+    int pool_rows;                 // rows of the pools' TMA view; this row reads zeros
+    unsigned *err;
+    uint64_t wait_limit_ns;
+    int inject_no_issue;           // testing: issue no copies so that waits run out
+};
+
+// Shared-memory plan (from a 1024-aligned base): Q tile, K ring, V ring, P
+// tile, then barriers, small state and the per-sequence unit prefix.
+template <int D>
+struct MqSmem {
+    static constexpr int kTileBytes = kMqTile * D * 2;   // K or V tile; Q (128 rows) too
+    static constexpr int kHalf = kMqTile * 128;          // one 128-byte column half of a tile
+    static constexpr int kPBytes = kMqRows * kMqTile * 2;
+    static constexpr int q = 0;
+    static constexpr int k = q + kTileBytes;
+    static constexpr int v = k + kMqKStages * kTileBytes;
+    static constexpr int p = v + kMqVStages * kTileBytes;
+    static constexpr int bars = p + kPBytes;
+    // barrier indices
+    static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kMqKStages,
+                         kVFull = kKEmpty + kMqKStages, kVEmpty = kVFull + kMqVStages, kSFull = kVEmpty + kMqVStages,
+                         kSFree = kSFull + 2, kPFull = kSFree + 2, kODone = kPFull + 1, kUnitFull = kODone + 1,
+                         kUnitEmpty = kUnitFull + 2, kDrain = kUnitEmpty + 2, kNumBars = kDrain + 1;
+    static constexpr int misc = bars + kNumBars * 8;     // [0..1] unit slots, [2] TMEM base, [3] abort
+    static constexpr int prefix = misc + 32;
+    static constexpr int bytes(int B) { return prefix + (B + 1) * 4 + 1024; }  // + base re-alignment
+};
+
+// A unit: rows = `tpb` consecutive query sources (chunk tokens, or members
+// of a sharing group) x the G heads of KV head kvh; K/V positions
+// [0, lim_max) read through table row trow; z0 = index of the unit's first
+// source in q's [sources][Hq][D] view.
+struct MqUnit {
+    int s, rb, kvh, nt, ctx, n, q0, lim_max, trow;
+};
+
+// Units of source s (0 for sources this kernel does not handle).
+__device__ __forceinline__ int mq_units_of(int s, const MqArgs &a) {
+    if (a.mode == kMqPrefix) {
+        const int n = __ldg(a.group_start + s + 1) - __ldg(a.group_start + s);
+        if (n < 1 || __ldg(a.group_len + s) <= 0)
+            return 0;
+        return ((n + a.tpb - 1) / a.tpb) * a.Hkv;
+    }
+    const int q0 = __ldg(a.query_start + s);
+    const int n = __ldg(a.query_start + s + 1) - q0;
+    const int c = __ldg(a.context_lens + s);
+    // decode tokens (n == 1) and inconsistent lengths are not this kernel's
+    if (n < 2 || c < n || (int64_t)c > a.mb * a.bs)
+        return 0;
+    return ((n + a.tpb - 1) / a.tpb) * a.Hkv;
+}
+
+__device__ __forceinline__ MqUnit mq_unit(int u, const int *prefix, const MqArgs &a) {
+    MqUnit U;
+    U.s = upper_bound_i(prefix, a.nsrc + 1, u) - 1;
+    if (a.mode == kMqPrefix) {
+        U.q0 = __ldg(a.group_start + U.s);
+        U.n = __ldg(a.group_start + U.s + 1) - U.q0;
+        U.ctx = __ldg(a.group_len + U.s);
+        U.trow = __ldg(a.group_ref + U.s);
+    } else {
+        U.q0 = __ldg(a.query_start + U.s);
+        U.n = __ldg(a.query_start + U.s + 1) - U.q0;
+        U.ctx = __ldg(a.context_lens + U.s);
+        U.trow = U.s;
+    }
+    const int nrb = (U.n + a.tpb - 1) / a.tpb;
+    const int idx = u - prefix[U.s];
+    U.rb = nrb - 1 - idx / a.Hkv;  // the longest causal ranges first
+    U.kvh = idx - (idx / a.Hkv) * a.Hkv;
+    U.lim_max = a.mode == kMqPrefix ? U.ctx : U.ctx - U.n + min(U.n, (U.rb + 1) * a.tpb);
+    U.nt = (U.lim_max + kMqTile - 1) / kMqTile;
+    return U;
+}
+
+// 2^x on the FMA and integer pipes, for part of the softmax exponentials so
+// that they do not all queue on the SFU (16 results per clock per SM): x =
+// n + f with n = round(x) (by the 1.5 * 2^23 add), f in [-1/2, 1/2]; 2^f by a
+// degree-4 polynomial (least-squares fit on Chebyshev nodes of [-1/2, 1/2],
+// relative error < 8e-6, coefficients from csrc/gen_exp2_poly.py); 2^n added
+// to the exponent field.  Arguments below -126 give 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+    const float xc = fmaxf(x, -126.f);
+    const float t = xc + 12582912.f;
+    const float f = xc - (t - 12582912.f);
+    float p = fmaf(f, 0.00927829f, 0.05586502f);
+    p = fmaf(p, f, 0.24030896f);
+    p = fmaf(p, f, 0.69312954f);
+    p = fmaf(p, f, 0.99999785f);
+    const float r = __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+    return x < -126.f ? 0.f : r;
+}
+
+__global__ void exp2_poly_test_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        y[i] = exp2_poly(x[i]);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B
+// both f16 or both bf16, A K-major, B K-major (b_mn = 0) or MN-major (1), N x
+// M = n x 128, optional negation of A.
+__host__ __device__ constexpr uint32_t mq_idesc(bool bf16, int n, bool negate_a, bool b_mn) {
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((negate_a ? 1u : 0u) << 13) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kMqRows >> 4) << 24);
+}
+
+// Bounded wait that also gives up when another role has aborted; a time-out
+// records the error and raises the abort flag.
+__device__ __forceinline__ bool mq_wait(uint32_t bar, uint32_t parity, const MqArgs &a, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag)
+            return false;
+        if (global_timer_ns() - t0 > a.wait_limit_ns) {
+            *abort_flag = 1;
+            atomicOr(a.err, kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// POLY: of every 8 pairs of a row's probabilities, POLY are computed with
+// exp2_poly and the rest with the SFU's exp2.
+template <int D, bool BF16, int POLY = 0>
+__global__ void __launch_bounds__(kMqThreads, 1)
+    mq_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const MqArgs a) {
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    using L = MqSmem<D>;
+    constexpr int KS = kMqKStages, VS = kMqVStages;
+    constexpr int NH = D / 64;              // 128-byte column halves of a row
+    constexpr int kTileBytes = L::kTileBytes;
+    constexpr int kHalf = L::kHalf;
+    constexpr uint32_t kTmemCols = 512;     // S0 | S1 | O
+    constexpr uint32_t kColO = 256;
+    constexpr unsigned FULL = 0xffffffffu;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sQ = base + L::q, sK = base + L::k, sV = base + L::v, sP = base + L::p;
+    auto bar = [&](int i) { return base + (uint32_t)(L::bars + i * 8); };
+    volatile int *misc = reinterpret_cast<volatile int *>(gbase + L::misc);
+    int *prefix = reinterpret_cast<int *>(gbase + L::prefix);
+    volatile int *abort_flag = misc + 3;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows_used = a.tpb * a.G;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(L::kQFull), 1);
+        mbar_init(bar(L::kQEmpty), 1);
+        for (int i = 0; i < KS; ++i) {
+            mbar_init(bar(L::kKFull + i), 1);
+            mbar_init(bar(L::kKEmpty + i), 1);
+        }
+        for (int i = 0; i < VS; ++i) {
+            mbar_init(bar(L::kVFull + i), 1);
+            mbar_init(bar(L::kVEmpty + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(L::kSFull + i), 1);
+            mbar_init(bar(L::kSFree + i), 4);      // one arrival per softmax warp
+            mbar_init(bar(L::kUnitFull + i), 1);
+            mbar_init(bar(L::kUnitEmpty + i), 5);  // the MMA thread + 4 softmax warps
+        }
+        mbar_init(bar(L::kPFull), 4);
+        mbar_init(bar(L::kODone), 1);
+        mbar_init(bar(L::kDrain), 1);
+        misc[3] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    // Q rows past tpb * G are never written by the TMA: keep them zero
+    for (int i = threadIdx.x; i < (kMqRows - rows_used) * 8 * NH; i += blockDim.x) {
+        const int r = rows_used + i / (8 * NH), rest = i % (8 * NH), h = rest / 8, c = rest % 8;
+        *reinterpret_cast<uint4 *>(gbase + L::q + h * kHalf + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    if (warp == 5) {
+        tmem_alloc(base + L::misc + 8, kTmemCols);
+        tmem_relinquish();
+    }
+
+    // every read of an input (and every write of out) comes after this
+    griddep_wait();
+    griddep_launch_dependents();
+
+    // ---- per-sequence unit counts and their prefix sums (block-wide scan)
+    {
+        const int nthr = blockDim.x;
+        const int per = (a.nsrc + nthr - 1) / nthr;
+        const int beg = min(a.nsrc, (int)threadIdx.x * per), end = min(a.nsrc, beg + per);
+        int local = 0;
+        for (int s = beg; s < end; ++s)
+            local += mq_units_of(s, a);
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        __shared__ int warp_tot[kMqThreads / 32];
+        if (lane == 31)
+            warp_tot[warp] = incl;
+        __syncthreads();
+        int run = 0;
+        for (int w = 0; w < warp; ++w)
+            run += warp_tot[w];
+        run += incl - local;
+        for (int s = beg; s < end; ++s) {
+            prefix[s] = run;
+            run += mq_units_of(s, a);
+        }
+        if (threadIdx.x == 0) {
+            int tot = 0;
+            for (int w = 0; w < kMqThreads / 32; ++w)
+                tot += warp_tot[w];
+            prefix[a.nsrc] = tot;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[2];
+    const int total = prefix[a.nsrc];
+
+    if (total > 0 && warp == 4) {
+        // ================= producer: unit scheduler + TMA loads =================
+        int k = 0;
+        uint32_t jg = 0;
+        int q_issued = -1;                 // last unit whose Q copy was issued
+        int k_last[KS], v_last[VS];        // last use index with copies issued, per stage
+        for (int i = 0; i < KS; ++i)
+            k_last[i] = -1;
+        for (int i = 0; i < VS; ++i)
+            v_last[i] = -1;
+        bool ok = true;
+        while (ok) {
+            int u = 0;
+            if (lane == 0)
+                u = atomicAdd(a.unit_counter, 1);
+            u = __shfl_sync(FULL, u, 0);
+            const int slot = k & 1;
+            ok = __all_sync(FULL, mq_wait(bar(L::kUnitEmpty + slot), ((k >> 1) & 1) ^ 1, a, abort_flag));
+            if (!ok)
+                break;
+            if (lane == 0) {
+                misc[slot] = u < total ? u : -1;
+                mbar_arrive(bar(L::kUnitFull + slot));
+            }
+            if (u >= total)
+                break;
+            const MqUnit U = mq_unit(u, prefix, a);
+            ok = __all_sync(FULL, mq_wait(bar(L::kQEmpty), (k & 1) ^ 1, a, abort_flag));
+            if (!ok)
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(L::kQFull), (uint32_t)(NH * rows_used * 128));
+                if (!a.inject_no_issue) {
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+                        tma_load_3d(sQ + h * kHalf, &tmQ, h * 64, U.kvh * a.G, U.q0 + U.rb * a.tpb, bar(L::kQFull));
+                    q_issued = k;
+                }
+            }
+            const int32_t *trow = a.block_tables + (size_t)U.trow * a.mb;
+            for (int j = 0; j < U.nt && ok; ++j, ++jg) {
+                // lanes 0..7: the pool row of each 16-position box of this tile;
+                // positions past the context (and bad table entries) read zeros
+                int y = a.pool_rows;
+                if (lane < kMqTile / 16) {
+                    const int pos = j * kMqTile + lane * 16;
+                    if (pos < U.ctx) {
+                        const int blk = __ldg(trow + pos / a.bs);
+                        if (blk < 0 || (int64_t)blk >= a.nb)
+                            atomicOr(a.err, kErrTable);
+                        else
+                            y = (blk * a.Hkv + U.kvh) * a.bs + pos % a.bs;
+                    }
+                }
+                const int st = (int)(jg % KS), vt = (int)(jg % VS);
+                ok = __all_sync(FULL, mq_wait(bar(L::kKEmpty + st), ((jg / KS) & 1) ^ 1, a, abort_flag));
+                if (!ok)
+                    break;
+                if (lane == 0)
+                    mbar_arrive_expect_tx(bar(L::kKFull + st), kTileBytes);
+                __syncwarp();
+                if (lane < kMqTile / 16 && !a.inject_no_issue) {
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+                        tma_load_2d(sK + st * kTileBytes + h * kHalf + lane * 2048, &tmK, h * 64, y,
+                                    bar(L::kKFull + st));
+                }
+                if (!a.inject_no_issue)
+                    k_last[st] = (int)(jg / KS);
+                ok = __all_sync(FULL, mq_wait(bar(L::kVEmpty + vt), ((jg / VS) & 1) ^ 1, a, abort_flag));
+                if (!ok)
+                    break;
+                if (lane == 0)
+                    mbar_arrive_expect_tx(bar(L::kVFull + vt), kTileBytes);
+                __syncwarp();
+                if (lane < kMqTile / 16 && !a.inject_no_issue) {
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+                        tma_load_2d(sV + vt * kTileBytes + h * kHalf + lane * 2048, &tmV, h * 64, y,
+                                    bar(L::kVFull + vt));
+                }
+                if (!a.inject_no_issue)
+                    v_last[vt] = (int)(jg / VS);
+            }
+            ++k;
+        }
+        // copies still in flight land before the CTA may exit (bounded)
+        if (lane == 0) {
+            if (q_issued >= 0)
+                mbar_wait_bounded(bar(L::kQFull), q_issued & 1, a.wait_limit_ns);
+            for (int i = 0; i < KS; ++i)
+                if (k_last[i] >= 0)
+                    mbar_wait_bounded(bar(L::kKFull + i), k_last[i] & 1, a.wait_limit_ns);
+            for (int i = 0; i < VS; ++i)
+                if (v_last[i] >= 0)
+                    mbar_wait_bounded(bar(L::kVFull + i), v_last[i] & 1, a.wait_limit_ns);
+        }
+        __syncwarp();
+    } else if (total > 0 && warp == 5) {
+        // ================= MMA issuer (one thread) =================
+        if (lane == 0) {
+            const uint32_t idesc_s = mq_idesc(BF16, kMqTile, a.negate_q != 0, false);
+            const uint32_t idesc_o = mq_idesc(BF16, D, false, true);
+            int k = 0;
+            uint32_t jg = 0;
+            bool ok = true, issued = false;
+            auto issue_pv = [&](uint32_t jp, bool first) {
+                const int vt = (int)(jp % VS);
+                if (!mq_wait(bar(L::kPFull), jp & 1, a, abort_flag) ||
+                    !mq_wait(bar(L::kVFull + vt), (jp / VS) & 1, a, abort_flag))
+                    return false;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kMqTile / 16; ++ks) {
+                    const uint64_t ad = smem_desc_sw128(sP + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(sV + vt * kTileBytes + ks * 2048, kHalf, 1024);
+                    tc_mma_ss(tmem + kColO, ad, bd, idesc_o, (first && ks == 0) ? 0u : 1u);
+                }
+                tc_commit(bar(L::kODone));
+                tc_commit(bar(L::kVEmpty + vt));
+                return true;
+            };
+            while (ok) {
+                const int slot = k & 1;
+                ok = mq_wait(bar(L::kUnitFull + slot), (k >> 1) & 1, a, abort_flag);
+                if (!ok)
+                    break;
+                const int u = misc[slot];
+                mbar_arrive(bar(L::kUnitEmpty + slot));
+                if (u < 0)
+                    break;
+                const MqUnit U = mq_unit(u, prefix, a);
+                ok = mq_wait(bar(L::kQFull), k & 1, a, abort_flag);
+                if (!ok)
+                    break;
+                for (int j = 0; j < U.nt; ++j, ++jg) {
+                    const int st = (int)(jg % KS);
+                    ok = mq_wait(bar(L::kKFull + st), (jg / KS) & 1, a, abort_flag) &&
+                         mq_wait(bar(L::kSFree + (jg & 1)), ((jg >> 1) & 1) ^ 1, a, abort_flag);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + (jg & 1) * kMqTile;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                        tc_mma_ss(d, smem_desc_sw128(sQ + off, 16, 1024),
+                                  smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(bar(L::kSFull + (jg & 1)));
+                    tc_commit(bar(L::kKEmpty + st));
+                    if (j == U.nt - 1)
+                        tc_commit(bar(L::kQEmpty));
+                    if (j >= 1 && !(ok = issue_pv(jg - 1, j == 1)))
+                        break;
+                }
+                if (!ok)
+                    break;
+                ok = issue_pv(jg - 1, U.nt == 1);
+                ++k;
+            }
+            // every MMA issued so far completes before TMEM is released
+            if (issued) {
+                tc_commit(bar(L::kDrain));
+                mbar_wait_bounded(bar(L::kDrain), 0, a.wait_limit_ns);
+            }
+        }
+        __syncwarp();
+    } else if (total > 0 && warp < 4) {
+        // ================= softmax + epilogue: thread r owns row r =================
+        const int r = threadIdx.x;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const int t = r / a.G, hj = r - (r / a.G) * a.G;
+        int k = 0;
+        uint32_t jg = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = k & 1;
+            ok = __all_sync(FULL, mq_wait(bar(L::kUnitFull + slot), (k >> 1) & 1, a, abort_flag));
+            if (!ok)
+                break;
+            const int u = misc[slot];
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(L::kUnitEmpty + slot));
+            if (u < 0)
+                break;
+            const MqUnit U = mq_unit(u, prefix, a);
+            const int tok = U.rb * a.tpb + t;  // the row's source within the unit's (chunk token / member)
+            const bool valid = r < rows_used && tok < U.n;
+            int lim = U.lim_max;
+            if (valid)
+                lim = a.mode == kMqPrefix ? min(__ldg(a.shared + U.q0 + tok), U.lim_max) : U.ctx - U.n + tok + 1;
+            float m_ref = -INFINITY, l = 0.f;
+            for (int j = 0; j < U.nt; ++j, ++jg) {
+                ok = __all_sync(FULL, mq_wait(bar(L::kSFull + (jg & 1)), (jg >> 1) & 1, a, abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                uint32_t sv[kMqTile];
+#pragma unroll
+                for (int c = 0; c < kMqTile / 32; ++c)
+                    tmem_ld32(lane_base + (jg & 1) * kMqTile + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(L::kSFree + (jg & 1)));
+                const int pos0 = j * kMqTile;
+                if (pos0 + kMqTile > lim) {
+#pragma unroll
+                    for (int i = 0; i < kMqTile; ++i)
+                        if (pos0 + i >= lim)
+                            sv[i] = __float_as_uint(-INFINITY);
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < kMqTile; i += 4) {
+                    mx0 = fmaxf(mx0, __uint_as_float(sv[i]));
+                    mx1 = fmaxf(mx1, __uint_as_float(sv[i + 1]));
+                    mx2 = fmaxf(mx2, __uint_as_float(sv[i + 2]));
+                    mx3 = fmaxf(mx3, __uint_as_float(sv[i + 3]));
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * a.scale_log2;
+                const float m_new = fmaxf(m_ref, mx);
+                const bool need = m_new > m_ref + kMqRescaleLog2;
+                float alpha = 1.f;
+                if (need) {
+                    alpha = exp2f(m_ref - m_new);
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+                const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;  // a row masked so far: P = 0
+                uint32_t pk[kMqTile / 2];
+                float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < kMqTile / 2; ++i) {
+                    const float x0 = fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, neg_m);
+                    const float x1 = fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, neg_m);
+                    const bool poly = (i & 7) < POLY;
+                    const float p0 = poly ? exp2_poly(x0) : exp2f(x0);
+                    const float p1 = poly ? exp2_poly(x1) : exp2f(x1);
+                    rs0 += p0;
+                    rs1 += p1;
+                    pk[i] = pack2<BF16>(p0, p1);
+                }
+                l += rs0 + rs1;
+                if (j > 0) {
+                    // P V of the previous tile is done: P may be overwritten and O rescaled
+                    ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    if (__any_sync(FULL, need)) {
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(lane_base + kColO + c * 32, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                            tmem_st32(lane_base + kColO + c * 32, o);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                // P -> shared memory, K-major 128-byte swizzle: positions
+                // 64h .. 64h+63 of row r at sP + h*kHalf + r*128, 16-byte chunk c
+                // at (c ^ (r % 8)) * 16
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t addr = sP + h * kHalf + r * 128 + ((c ^ (r & 7)) << 4);
+                        const int b = h * 32 + c * 4;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[b]),
+                                     "r"(pk[b + 1]), "r"(pk[b + 2]), "r"(pk[b + 3])
+                                     : "memory");
+                    }
+                if (pos0 + kMqTile > U.ctx) {
+                    // V rows at positions >= ctx are unwritten (or poisoned) slots
+                    const int vt = (int)(jg % VS);
+                    ok = __all_sync(FULL, mq_wait(bar(L::kVFull + vt), (jg / VS) & 1, a, abort_flag));
+                    if (!ok)
+                        break;
+                    if (pos0 + r >= U.ctx) {
+#pragma unroll
+                        for (int h = 0; h < NH; ++h)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t addr = sV + vt * kTileBytes + h * kHalf + r * 128 + c * 16;
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
+                                             : "memory");
+                            }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(L::kPFull));
+            }
+            if (!ok)
+                break;
+            // ---- epilogue: O / l of every valid row
+            ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
+            if (!ok)
+                break;
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t orow_idx = (size_t)(U.q0 + (valid ? tok : 0)) * a.Hq + U.kvh * a.G + hj;
+            uint16_t *orow = a.out + orow_idx * D;
+            if (a.mode == kMqPrefix && valid) {
+                a.part_m[orow_idx] = m_ref;
+                a.part_l[orow_idx] = l;
+            }
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + kColO + c * 32, o);
+                tmem_wait_ld();
+                if (a.mode == kMqPrefix) {
+                    // unnormalized fp32 partial, relative to 2^m_ref
+                    if (valid) {
+                        float4 *dst = reinterpret_cast<float4 *>(a.part_o + orow_idx * D + c * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            dst[v4] = make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
+                                                  __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
+                    }
+                } else if (valid) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 w;
+                        w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * inv, __uint_as_float(o[v4 * 8 + 1]) * inv);
+                        w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * inv, __uint_as_float(o[v4 * 8 + 3]) * inv);
+                        w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * inv, __uint_as_float(o[v4 * 8 + 5]) * inv);
+                        w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * inv, __uint_as_float(o[v4 * 8 + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(orow + c * 32 + v4 * 8) = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            ++k;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5)
+        tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace pkv
+
+namespace pkv {
+
+// Preparation of a shared-prefix decode step (one CTA).  For every sequence
+// the defaults (no shared prefix: whole context left to the decode kernel);
+// then one warp per sharing group: the reference member (the first with the
+// largest claimed shared length), each member's effective shared length --
+// its claim, capped so that its last position stays in its own blocks, and
+// cut at the first table entry that differs from the reference's -- the
+// group's longest, and each member's remaining length and table offset for
+// the decode kernel.  A claim that does not hold only shrinks the shared
+// part, so the result stays exact.
+__global__ void __launch_bounds__(1024) cascade_prep_kernel(
+    const int32_t *__restrict__ group_start, int NG, const int32_t *__restrict__ claimed,
+    const int32_t *__restrict__ context_lens, const int32_t *__restrict__ block_tables, int64_t mb, int bs,
+    int B, int32_t *group_ref, int32_t *group_len, int32_t *shared, int32_t *suffix_len, int32_t *table_off,
+    int *mq_counter, unsigned *err) {
+    constexpr unsigned FULL = 0xffffffffu;
+    griddep_wait();
+    if (threadIdx.x == 0)
+        *mq_counter = 0;
+    const int64_t cap = mb * bs;
+    auto ctx_of = [&](int s) {
+        const int c = __ldg(context_lens + s);
+        if (c < 0 || (int64_t)c > cap) {
+            atomicOr(err, kErrContext);
+            return c < 0 ? 0 : (int)cap;
+        }
+        return c;
+    };
+    for (int s = threadIdx.x; s < B; s += blockDim.x) {
+        shared[s] = 0;
+        suffix_len[s] = ctx_of(s);
+        table_off[s] = 0;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warps = blockDim.x >> 5;
+    for (int g = threadIdx.x >> 5; g < NG; g += warps) {
+        int gs = __ldg(group_start + g), ge = __ldg(group_start + g + 1);
+        if (gs < 0 || ge > B || ge < gs) {
+            if (lane == 0)
+                atomicOr(err, kErrContext);
+            gs = ge = 0;
+        }
+        // claims in whole blocks, the sequence's last position kept private
+        auto claim_blocks = [&](int m) {
+            const int c = ctx_of(m);
+            const int cl = __ldg(claimed + m);
+            if (c < 1 || cl <= 0)
+                return 0;
+            return min(cl, c - 1) / bs;
+        };
+        int best = -1, best_c = -1;
+        for (int m = gs + lane; m < ge; m += 32) {
+            const int c = claim_blocks(m);
+            if (c > best_c) {
+                best_c = c;
+                best = m;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const int oc = __shfl_xor_sync(FULL, best_c, o), om = __shfl_xor_sync(FULL, best, o);
+            if (oc > best_c || (oc == best_c && om >= 0 && (best < 0 || om < best))) {
+                best_c = oc;
+                best = om;
+            }
+        }
+        const int ref = best < 0 ? gs : best;
+        const int ref_blocks = best_c < 0 ? 0 : best_c;
+        const int32_t *tr = block_tables + (size_t)ref * mb;
+        int glen = 0;
+        for (int m = gs + lane; m < ge; m += 32) {
+            const int cb = min(claim_blocks(m), ref_blocks);
+            const int32_t *tm = block_tables + (size_t)m * mb;
+            int e = 0;
+            while (e < cb && __ldg(tm + e) == __ldg(tr + e))
+                ++e;
+            shared[m] = e * bs;
+            suffix_len[m] = ctx_of(m) - e * bs;
+            table_off[m] = e;
+            glen = max(glen, e * bs);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            glen = max(glen, __shfl_xor_sync(FULL, glen, o));
+        if (lane == 0) {
+            group_ref[g] = ref;
+            group_len[g] = glen;
+        }
+    }
+}
+
+}  // namespace pkv

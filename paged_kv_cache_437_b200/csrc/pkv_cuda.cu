@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "decode.cuh"
+#include "mq_attention.cuh"
 #include "pkv.h"
 
 namespace pkv {
@@ -151,6 +152,24 @@ bool make_pool_map_uncached(CUtensorMap *map, const pkv_cache &c) {
     CUresult r = fn(map, dt, 2, c.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The query rows of a chunked-prefill call, q [T][Hq][D], as a 3-D tensor
+// (columns, heads, tokens); one box = 64 columns x G heads x tpb tokens
+// (128-byte swizzle), i.e. the rows (token, head of the group) of one unit
+// of the multi-query kernel, one 128-byte column half at a time.
+bool make_q_map(CUtensorMap *map, const void *q, int64_t T, int64_t Hq, int64_t D, int G, int tpb, bool bf16) {
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)(Hq * D * 2)};
+    cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)tpb};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                    const_cast<void *>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -403,6 +422,57 @@ WsLayout ws_layout(const Plan &p, int64_t B, int64_t Hq, int64_t D, int64_t max_
     return w;
 }
 
+// Launch the multi-query kernel.  Prefill: every chunk of two or more tokens
+// (the expansion kernel has zeroed its unit counter and given those tokens
+// no decode work).  Prefix: every sharing group's common prefix (the cascade
+// preparation kernel has zeroed the counter and filled the group arrays).
+// One CTA per SM, programmatic stream serialisation.
+pkv_status mq_launch(MqArgs a, const void *q, int64_t nz, const pkv_cache &kc, const pkv_cache &vc, float scale,
+                     pkv_stream stream) {
+    const int64_t Hkv = kc.num_kv_heads, D = kc.head_dim;
+    a.Hkv = (int)Hkv;
+    a.G = (int)(a.Hq / Hkv);
+    a.tpb = kMqRows / a.G;
+    a.nb = kc.num_blocks;
+    a.bs = (int)kc.block_size;
+    a.scale_log2 = std::fabs(scale) * 1.4426950408889634f;
+    a.negate_q = scale < 0.0f ? 1 : 0;
+    a.pool_rows = (int)(kc.num_blocks * Hkv * kc.block_size);
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.inject_no_issue = g_inject_no_issue;
+    const bool bf16 = kc.dtype == PKV_BF16;
+    CUtensorMap tmQ, tmK, tmV;
+    if (!make_q_map(&tmQ, q, nz, a.Hq, D, a.G, a.tpb, bf16) || !make_pool_map(&tmK, kc) || !make_pool_map(&tmV, vc))
+        return PKV_ERR_CUDA;
+    void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const MqArgs) = nullptr;
+    int smem = 0;
+    // PKV_MQ_POLY=1: 3 of every 8 probability pairs by the FMA-pipe exp2
+    const bool poly = env_int("PKV_MQ_POLY", 0) == 1;
+    if (D == 128) {
+        if (poly)
+            k = bf16 ? mq_attention_kernel<128, true, 3> : mq_attention_kernel<128, false, 3>;
+        else
+            k = bf16 ? mq_attention_kernel<128, true> : mq_attention_kernel<128, false>;
+        smem = MqSmem<128>::bytes(a.nsrc);
+    } else {
+        k = bf16 ? mq_attention_kernel<64, true> : mq_attention_kernel<64, false>;
+        smem = MqSmem<64>::bytes(a.nsrc);
+    }
+    // one CTA per SM: a second one would only wait for the first's TMEM
+    smem = std::max(smem, kMaxSmemPerCta / 2 + 1024);
+    if (smem > kMaxSmemPerCta)
+        return PKV_ERR_INVALID;
+    if (!cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta)))
+        return PKV_ERR_CUDA;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (!cuda_ok(launch_dependent(k, dim3(sms), dim3(kMqThreads), smem, (cudaStream_t)stream, tmQ, tmK, tmV, a)))
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
 }  // namespace
 }  // namespace pkv
 
@@ -496,12 +566,18 @@ struct FusedAppend {
     const int64_t *slots;
 };
 
+// Shared-prefix cascade inputs of the decode kernel (see DecodeArgs).
+struct CascadeIn {
+    const int32_t *table_offset;
+    const float *init_o, *init_m, *init_l;
+};
+
 pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv_cache k_cache,
                        pkv_cache v_cache, const int32_t *block_tables, int64_t max_blocks_per_seq,
                        const int32_t *context_lens, float scale, void *out, void *workspace,
                        size_t workspace_bytes, int32_t partition_tokens, pkv_stream stream,
                        const FusedAppend *fa, const int32_t *table_rows = nullptr,
-                       pkv_dtype q_dtype = PKV_F16) {
+                       pkv_dtype q_dtype = PKV_F16, const CascadeIn *cas = nullptr) {
     if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0)
         return PKV_ERR_INVALID;
     const bool fp8 = k_cache.dtype == PKV_E4M3;
@@ -601,6 +677,12 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.v_cache = static_cast<uint16_t *>(v_cache.data);
     a.pool_slots = k_cache.num_blocks * bs;
     a.table_rows = table_rows;
+    a.table_offset = cas ? cas->table_offset : nullptr;
+    a.init_o = cas ? cas->init_o : nullptr;
+    a.init_m = cas ? cas->init_m : nullptr;
+    a.init_l = cas ? cas->init_l : nullptr;
+    if (cas && (fp8 || p.fma))
+        return PKV_ERR_INVALID;  // the cascade resumes 16-bit MMA accumulators only
     a.k_scales = k_cache.scales;
     a.v_scales = v_cache.scales;
 
@@ -695,7 +777,8 @@ size_t pkv_prefill_workspace_bytes(int64_t num_tokens, int64_t num_q_heads, int6
                                                   max_context_len, PKV_PARTITION_AUTO);
     if (dec == 0 && num_tokens > 0)
         return 0;
-    return align256((size_t)num_tokens * 8) + dec;
+    // per-token lengths and table rows, then the multi-query unit counter
+    return align256((size_t)num_tokens * 8 + 4) + dec;
 }
 
 pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_seqs, int64_t num_q_heads,
@@ -710,24 +793,169 @@ pkv_status pkv_prefill_attention(const void *q, int64_t num_tokens, int64_t num_
     if (num_seqs == 0 || !query_start || !context_lens || !workspace || !aligned16(workspace) ||
         !cache_ok(k_cache) || (reinterpret_cast<uintptr_t>(query_start) & 3u))
         return PKV_ERR_INVALID;
-    const size_t head = align256((size_t)num_tokens * 8);
+    const size_t head = align256((size_t)num_tokens * 8 + 4);
     if (workspace_bytes < head)
         return PKV_ERR_INVALID;
     unsigned *err = error_word();
     if (!err)
         return PKV_ERR_CUDA;
+    const int64_t Hkv = k_cache.num_kv_heads, D = k_cache.head_dim;
+    const int64_t G = Hkv > 0 ? num_q_heads / Hkv : 0;
+    // Chunks of two or more tokens run on the multi-query tensor-core kernel
+    // (one K/V pass per block of tokens); decode tokens stay on the decode
+    // kernel.  PKV_PREFILL_MQ=0 sends every token through the decode kernel.
+    const bool mq = env_int("PKV_PREFILL_MQ", 1) != 0 && (D == 64 || D == 128) && G >= 1 && G <= kMqRows &&
+                    num_q_heads % Hkv == 0 && scale != 0.0f && std::isfinite(scale) &&
+                    num_seqs <= kMqMaxSeqs && q && out && aligned16(q) && aligned16(out) && block_tables &&
+                    (reinterpret_cast<uintptr_t>(block_tables) & 3u) == 0 && same_shape(k_cache, v_cache) &&
+                    cache_ok(v_cache) && k_cache.block_size % kTileTokens == 0 &&
+                    k_cache.num_blocks * Hkv * k_cache.block_size < (int64_t(1) << 31) - 16 &&
+                    max_blocks_per_seq > 0 && max_blocks_per_seq * k_cache.block_size < (int64_t(1) << 30);
     int32_t *lens = static_cast<int32_t *>(workspace);
     int32_t *rows = lens + num_tokens;
+    int *counter = reinterpret_cast<int *>(rows + num_tokens);
     const int64_t blocks = std::min<int64_t>((num_tokens + 255) / 256, 148 * 8);
     prefill_expand_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
         query_start, context_lens, (int)num_seqs, (int)num_tokens, max_blocks_per_seq * k_cache.block_size,
-        lens, rows, err);
+        lens, rows, mq ? counter : nullptr, err);
     if (!cuda_ok(cudaGetLastError()))
         return PKV_ERR_CUDA;
     char *rest = static_cast<char *>(workspace) + head;
-    return decode_impl(q, num_tokens, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq, lens,
-                       scale, out, workspace_bytes > head ? rest : nullptr, workspace_bytes - head,
-                       PKV_PARTITION_AUTO, stream, nullptr, rows);
+    pkv_status st = decode_impl(q, num_tokens, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                lens, scale, out, workspace_bytes > head ? rest : nullptr, workspace_bytes - head,
+                                PKV_PARTITION_AUTO, stream, nullptr, rows);
+    if (st != PKV_OK || !mq)
+        return st;
+    MqArgs a = {};
+    a.mode = kMqPrefill;
+    a.out = static_cast<uint16_t *>(out);
+    a.block_tables = block_tables;
+    a.query_start = query_start;
+    a.context_lens = context_lens;
+    a.nsrc = (int)num_seqs;
+    a.mb = max_blocks_per_seq;
+    a.B = (int)num_seqs;
+    a.T = (int)num_tokens;
+    a.Hq = (int)num_q_heads;
+    a.unit_counter = counter;
+    a.err = err;
+    return mq_launch(a, q, num_tokens, k_cache, v_cache, scale, stream);
+}
+
+// Workspace of pkv_append_decode_attention_shared_prefix:
+//   group_ref [NG] | group_len [NG] | shared [B] | suffix_len [B] | table_off [B] | counter  (256-aligned)
+//   part_o [B][Hq][D] f32 | part_m [B][Hq] | part_l [B][Hq]                                  (each 256-aligned)
+//   then the decode kernel's AUTO workspace.
+struct CascadeWs {
+    size_t ref = 0, len = 0, shared = 0, suffix = 0, toff = 0, counter = 0, o = 0, m = 0, l = 0, dec = 0, total = 0;
+};
+
+static CascadeWs cascade_ws(int64_t B, int64_t Hq, int64_t D, int64_t NG, size_t dec_bytes) {
+    CascadeWs w;
+    w.ref = 0;
+    w.len = w.ref + NG * 4;
+    w.shared = w.len + NG * 4;
+    w.suffix = w.shared + B * 4;
+    w.toff = w.suffix + B * 4;
+    w.counter = w.toff + B * 4;
+    w.o = align256(w.counter + 4);
+    w.m = align256(w.o + (size_t)B * Hq * D * 4);
+    w.l = align256(w.m + (size_t)B * Hq * 4);
+    w.dec = align256(w.l + (size_t)B * Hq * 4);
+    w.total = w.dec + dec_bytes;
+    return w;
+}
+
+size_t pkv_shared_prefix_workspace_bytes(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                         int64_t head_dim, int64_t max_context_len, int64_t num_groups) {
+    if (num_seqs < 0 || num_groups < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+        (head_dim != 64 && head_dim != 128) || max_context_len < 0)
+        return 0;
+    const size_t dec = pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                                  PKV_PARTITION_AUTO);
+    return cascade_ws(num_seqs, num_q_heads, head_dim, num_groups, dec).total;
+}
+
+pkv_status pkv_append_decode_attention_shared_prefix(
+    const void *k_new, const void *v_new, const int64_t *slot_mapping, const void *q, int64_t num_seqs,
+    int64_t num_q_heads, pkv_cache k_cache, pkv_cache v_cache, const int32_t *block_tables,
+    int64_t max_blocks_per_seq, const int32_t *context_lens, const int32_t *group_start, int64_t num_groups,
+    const int32_t *shared_lens, float scale, void *out, void *workspace, size_t workspace_bytes,
+    pkv_stream stream) {
+    const bool append = k_new || v_new || slot_mapping;
+    if (append && num_seqs > 0 &&
+        (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new) ||
+         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u)))
+        return PKV_ERR_INVALID;
+    if (num_seqs < 0 || num_groups < 0 || num_groups > kMqMaxSeqs || num_q_heads <= 0)
+        return PKV_ERR_INVALID;
+    if (!cache_ok(k_cache) || !cache_ok(v_cache) || !same_shape(k_cache, v_cache))
+        return PKV_ERR_INVALID;
+    const int64_t Hkv = k_cache.num_kv_heads, D = k_cache.head_dim;
+    if (num_q_heads % Hkv != 0 || num_q_heads / Hkv > kMqRows || (D != 64 && D != 128) || !std::isfinite(scale))
+        return PKV_ERR_INVALID;
+    if (num_seqs == 0)
+        return PKV_OK;
+    if (num_groups > 0 && (!group_start || !shared_lens || (reinterpret_cast<uintptr_t>(group_start) & 3u) ||
+                           (reinterpret_cast<uintptr_t>(shared_lens) & 3u)))
+        return PKV_ERR_INVALID;
+    if (!workspace || !aligned16(workspace) || !block_tables || !context_lens || !q || !aligned16(q))
+        return PKV_ERR_INVALID;
+    const size_t dec = pkv_decode_workspace_bytes(num_seqs, num_q_heads, Hkv, D, max_blocks_per_seq * k_cache.block_size,
+                                                  PKV_PARTITION_AUTO);
+    const CascadeWs wl = cascade_ws(num_seqs, num_q_heads, D, num_groups, dec);
+    if (workspace_bytes < wl.total)
+        return PKV_ERR_INVALID;
+    char *ws = static_cast<char *>(workspace);
+    const FusedAppend fa{k_new, v_new, slot_mapping};
+    if (num_groups == 0 || scale == 0.0f) {
+        // nothing shared (or a degenerate scale): the plain decode step
+        return decode_impl(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           context_lens, scale, out, dec ? ws + wl.dec : nullptr, dec, PKV_PARTITION_AUTO, stream,
+                           append ? &fa : nullptr);
+    }
+    unsigned *err = error_word();
+    if (!err)
+        return PKV_ERR_CUDA;
+    int32_t *g_ref = reinterpret_cast<int32_t *>(ws + wl.ref);
+    int32_t *g_len = reinterpret_cast<int32_t *>(ws + wl.len);
+    int32_t *shared = reinterpret_cast<int32_t *>(ws + wl.shared);
+    int32_t *suffix = reinterpret_cast<int32_t *>(ws + wl.suffix);
+    int32_t *toff = reinterpret_cast<int32_t *>(ws + wl.toff);
+    int *counter = reinterpret_cast<int *>(ws + wl.counter);
+    float *po = reinterpret_cast<float *>(ws + wl.o);
+    float *pm = reinterpret_cast<float *>(ws + wl.m);
+    float *pl = reinterpret_cast<float *>(ws + wl.l);
+    cascade_prep_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(
+        group_start, (int)num_groups, shared_lens, context_lens, block_tables, max_blocks_per_seq,
+        (int)k_cache.block_size, (int)num_seqs, g_ref, g_len, shared, suffix, toff, counter, err);
+    if (!cuda_ok(cudaGetLastError()))
+        return PKV_ERR_CUDA;
+    MqArgs a = {};
+    a.mode = kMqPrefix;
+    a.out = nullptr;
+    a.block_tables = block_tables;
+    a.group_start = group_start;
+    a.group_ref = g_ref;
+    a.group_len = g_len;
+    a.shared = shared;
+    a.part_o = po;
+    a.part_m = pm;
+    a.part_l = pl;
+    a.nsrc = (int)num_groups;
+    a.mb = max_blocks_per_seq;
+    a.B = (int)num_seqs;
+    a.T = (int)num_seqs;
+    a.Hq = (int)num_q_heads;
+    a.unit_counter = counter;
+    a.err = err;
+    pkv_status st = mq_launch(a, q, num_seqs, k_cache, v_cache, scale, stream);
+    if (st != PKV_OK)
+        return st;
+    const CascadeIn cas{toff, po, pm, pl};
+    return decode_impl(q, num_seqs, num_q_heads, k_cache, v_cache, block_tables, max_blocks_per_seq, suffix, scale,
+                       out, dec ? ws + wl.dec : nullptr, dec, PKV_PARTITION_AUTO, stream, append ? &fa : nullptr,
+                       nullptr, PKV_F16, &cas);
 }
 
 pkv_status pkv_decode_attention_e4m3(const void *q, pkv_dtype q_dtype, int64_t num_seqs, int64_t num_q_heads,
@@ -798,6 +1026,16 @@ pkv_status pkv_get_last_error(void) {
         return (v & kErrTimeout) ? PKV_ERR_TIMEOUT : PKV_ERR_DEVICE_CHECK;
     }
     return PKV_OK;
+}
+
+pkv_status pkv_test_exp2_poly(const float *x, float *y, int64_t n, pkv_stream stream) {
+    if (n < 0 || (n > 0 && (!x || !y)))
+        return PKV_ERR_INVALID;
+    if (n == 0)
+        return PKV_OK;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
+    exp2_poly_test_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+    return cuda_ok(cudaGetLastError()) ? PKV_OK : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_test_inject_wait_timeout(int32_t enable, int64_t wait_limit_ns) {

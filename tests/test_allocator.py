@@ -250,3 +250,38 @@ def test_batch_copy_on_write():
         full.append_slots_cow([k1, k2])    # needs two fresh blocks, one is free
     assert e.value.status == pkv.PKV_ERR_OOM
     assert full.context_len(k1) == 20 and full.context_len(k2) == 20
+
+
+def test_batch_prefix_groups():
+    bs = 16
+    a = pkv.BlockAllocator(64, bs)
+    p1 = a.seq_create()
+    for _ in range(3 * bs + 5):
+        a.append_slot(p1)
+    m1 = a.seq_fork(p1, 3)
+    m2 = a.seq_fork(p1, 2)
+    for _ in range(bs + 1):
+        a.append_slot(m1)
+        a.append_slot(m2)
+    lone = a.seq_create()
+    for _ in range(2 * bs):
+        a.append_slot(lone)
+    p2 = a.seq_create()
+    for _ in range(bs):
+        a.append_slot(p2)
+    m3 = a.seq_fork(p2, 1)
+    a.append_slot(m3)
+    # groups: runs of consecutive sequences whose first block is one shared block
+    starts, shared = a.prefix_groups([p1, m1, m2, lone, m3, p2])
+    assert starts.tolist() == [0, 3, 4, 6]
+    # claims: leading blocks with refcount > 1, times bs (p1's third block is
+    # shared with m1 only; its fourth is private)
+    assert shared.tolist() == [3 * bs, 3 * bs, 2 * bs, 0, bs, bs]
+    # a shared sequence separated from its group starts a new one
+    starts, _ = a.prefix_groups([m1, lone, m2])
+    assert starts.tolist() == [0, 1, 2, 3]
+    starts, shared = a.prefix_groups([])
+    assert starts.tolist() == [0] and shared.size == 0
+    with pytest.raises(pkv.PkvError):
+        a.prefix_groups([p1, 999])
+    a.close()

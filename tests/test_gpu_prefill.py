@@ -22,10 +22,12 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{workloads.DTYPE_NAMES[c[0]]}_{c[1]}_{c[2]}_{c[3]}_bs{c[4]}")
-def test_prefill_matches_oracle(case):
+def _run_case(case, seed=None, scale=None, expect=pkv.PKV_OK):
+    """Build one mixed batch, run pkv_prefill_attention on it and the fp64
+    oracle on the same inputs; returns (GPU out, oracle out, K/V pools after
+    the append on both sides)."""
     dtype, hq, hkv, d, bs, seqs = case
-    rng = np.random.default_rng(70 + len(seqs))
+    rng = np.random.default_rng(70 + len(seqs) if seed is None else seed)
     ctx = np.array([c for c, _ in seqs], dtype=np.int32)
     nq = np.array([n for _, n in seqs], dtype=np.int32)
     qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
@@ -52,7 +54,8 @@ def test_prefill_matches_oracle(case):
     slots = np.concatenate([oracle.slot_mapping(np.repeat(tables[s:s + 1], nq[s], axis=0),
                                                 np.arange(ctx[s] - nq[s], ctx[s]), bs)
                             for s in range(len(seqs))]).astype(np.int64)
-    scale = float(np.float32(1.0) / np.sqrt(np.float32(d)))
+    if scale is None:
+        scale = float(np.float32(1.0) / np.sqrt(np.float32(d)))
 
     k_ref, v_ref = kc.copy(), vc.copy()
     oracle.append(k_ref, kn, slots)
@@ -62,14 +65,67 @@ def test_prefill_matches_oracle(case):
     kd, vd = gh.dev(kc, dtype), gh.dev(vc, dtype)
     pkv.pkv_append(gh.dev(kn, dtype), gh.dev(vn, dtype), torch.from_numpy(slots).cuda(), kd, vd)
     qd = gh.dev(q, dtype)
-    out = torch.empty_like(qd)
+    out = torch.full_like(qd, float("nan"))
     ws = torch.empty(pkv.pkv_prefill_workspace_bytes(t, hq, hkv, d, mb * bs), dtype=torch.uint8, device="cuda")
     pkv.pkv_prefill_attention(qd, kd, vd, torch.from_numpy(tables).cuda(), torch.from_numpy(qs).cuda(),
                               torch.from_numpy(ctx).cuda(), scale, out, ws)
     torch.cuda.synchronize()
-    assert pkv.pkv_get_last_error() == pkv.PKV_OK
-    assert np.array_equal(gh.host_bits(kd), k_ref) and np.array_equal(gh.host_bits(vd), v_ref)
-    gh.assert_close(gh.to_f64(out), ref, dtype, "prefill")
+    st = pkv.pkv_get_last_error()
+    assert st == expect, pkv.pkv_status_string(st)
+    return out, ref, (gh.host_bits(kd), gh.host_bits(vd)), (k_ref, v_ref)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{workloads.DTYPE_NAMES[c[0]]}_{c[1]}_{c[2]}_{c[3]}_bs{c[4]}")
+def test_prefill_matches_oracle(case):
+    out, ref, pools, pools_ref = _run_case(case)
+    assert np.array_equal(pools[0], pools_ref[0]) and np.array_equal(pools[1], pools_ref[1])
+    gh.assert_close(gh.to_f64(out), ref, case[0], "prefill")
+
+
+# the multi-query tensor-core kernel's edge cases: chunks that are not a
+# multiple of the row block, tails whose last tile runs past the context
+# (V rows there are poisoned), one-tile and many-tile ranges, several chunks
+# in one call, a chunk that is the whole context, the largest GQA group
+MQ_CASES = [
+    (BF16, 64, 8, 128, 16, [(129, 129), (4000, 300), (1, 1), (257, 2)]),
+    (F16, 16, 4, 128, 32, [(1000, 999), (77, 3), (128, 128), (129, 1)]),
+    (BF16, 128, 1, 128, 16, [(300, 20), (16, 16)]),
+    (F16, 4, 4, 64, 32, [(700, 256), (255, 255), (90, 7)]),
+    (BF16, 24, 8, 64, 16, [(513, 64), (2048, 1), (40, 40)]),
+]
+
+
+@pytest.mark.parametrize("case", MQ_CASES, ids=lambda c: f"{workloads.DTYPE_NAMES[c[0]]}_{c[1]}_{c[2]}_{c[3]}_bs{c[4]}")
+def test_multi_query_kernel_edge_cases(case):
+    out, ref, _, _ = _run_case(case, seed=5)
+    gh.assert_close(gh.to_f64(out), ref, case[0], "prefill (multi-query kernel)")
+
+
+def test_negative_scale():
+    case = (F16, 32, 8, 128, 16, [(600, 200), (50, 1)])
+    out, ref, _, _ = _run_case(case, seed=6, scale=-0.07)
+    gh.assert_close(gh.to_f64(out), ref, F16, "prefill, negative scale")
+
+
+def test_multi_query_kernel_matches_the_per_token_path(monkeypatch):
+    case = (BF16, 64, 8, 128, 16, [(1500, 400), (300, 1)])
+    out_mq, ref, _, _ = _run_case(case, seed=7)
+    monkeypatch.setenv("PKV_PREFILL_MQ", "0")
+    out_tok, _, _, _ = _run_case(case, seed=7)
+    gh.assert_close(gh.to_f64(out_mq), ref, BF16, "multi-query kernel")
+    gh.assert_close(gh.to_f64(out_tok), ref, BF16, "per-token decode path")
+
+
+def test_multi_query_wait_timeout_is_reported_and_recovers():
+    case = (BF16, 64, 8, 128, 16, [(700, 300)])
+    pkv.pkv_test_inject_wait_timeout(True, 20_000_000)   # 20 ms
+    try:
+        _run_case(case, seed=8, expect=pkv.PKV_ERR_TIMEOUT)
+    finally:
+        pkv.pkv_test_inject_wait_timeout(False)
+    assert pkv.pkv_get_last_error() == pkv.PKV_OK  # read and cleared above
+    out, ref, _, _ = _run_case(case, seed=8)
+    gh.assert_close(gh.to_f64(out), ref, BF16, "prefill after a time-out")
 
 
 def test_prefill_flags_inconsistent_lengths():
