@@ -291,8 +291,9 @@ size_t pkv_prefill_workspace_bytes(int64_t num_tokens, int64_t num_q_heads, int6
  * within its claim, (b) end before its last position (the position of this
  * step's new token stays in the sequence's own block) and (c) have the same
  * table entries as the reference's: a wrong claim only shrinks the shared
- * part, never changes the result.  An invalid group_start entry is flagged
- * (PKV_ERR_DEVICE_CHECK) and that group computed without sharing.
+ * part, never changes the result.  A group_start that does not run from 0
+ * to B without decreasing is flagged (PKV_ERR_DEVICE_CHECK) and the step
+ * computed without sharing (still exact).
  * Limits: those of pkv_decode_attention, 16-bit pools, G <= 128,
  * num_groups <= 4096; num_groups == 0 (or scale == 0) runs the plain step.
  * ------------------------------------------------------------------------ */

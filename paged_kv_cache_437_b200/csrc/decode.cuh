@@ -316,12 +316,15 @@ __device__ __forceinline__ void sts_f4(uint32_t addr, float x, float y, float z,
 // shared memory and the MMAs run in f16 (a bf16 query is converted to f16,
 // exact in f16's normal range); K scales multiply the scores, V scales the
 // probabilities.
-template <int D, bool BF16, int NT, bool FP8 = false, bool FMA = false>
+// CAS: the shared-prefix cascade (table offsets, resume from a partial);
+// compiled separately so that the plain decode is unchanged by it.
+template <int D, bool BF16, int NT, bool FP8 = false, bool FMA = false, bool CAS = false>
 __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(!FMA || (!FP8 && NT == 1), "the CUDA-core variant: 16-bit pools, 8 heads per unit");
+    static_assert(!CAS || (!FP8 && !FMA), "the cascade resumes 16-bit MMA accumulators");
     constexpr int kTile = kTileTokens * D * 2;  // bytes of one 16-bit K (or V) tile
     constexpr int kMT = D / 16;                 // k-steps of Q K^T == 16-row d tiles of P V
     constexpr int HPU = 8 * NT;                 // query heads per unit (MMA N)
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         for (int s = blockIdx.x; s < a.B; s += gridDim.x) {
             if (ctxs[s] != 0)
                 continue;
-            if (!FP8 && !FMA && a.init_l && a.table_offset && __ldg(a.table_offset + s) > 0) {
+            if (CAS && __ldg(a.table_offset + s) > 0) {
                 // nothing after the shared prefix: its partial, normalized
                 uint32_t *o = reinterpret_cast<uint32_t *>(a.out + (size_t)s * a.Hq * D);
                 for (int i = threadIdx.x; i < a.Hq * D / 2; i += blockDim.x) {
@@ -491,7 +494,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const int nblk = ceil_div_i(ns.ctx, a.bs);
             nx_seq = ns.seq;
             nx_base = lb;
-            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.trow * a.mb + ns.toff + lb + lane) : 0;
+            nx_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ns.trow * a.mb + (CAS ? ns.toff : 0) + lb + lane) : 0;
         }
     };
     // set when the producer enters a unit; the prefetch for the unit after it
@@ -510,7 +513,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 nx_seq = -1;
             } else {
                 const int nblk = ceil_div_i(ps.ctx, a.bs);
-                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.trow * a.mb + ps.toff + lb + lane) : 0;
+                tb_val = (lb + lane < nblk) ? __ldg(a.block_tables + (size_t)ps.trow * a.mb + (CAS ? ps.toff : 0) + lb + lane) : 0;
             }
         }
         if (want_prefetch) {
@@ -685,8 +688,8 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             l_run[nt][0] = l_run[nt][1] = 0.f;
         }
 
-        if constexpr (!FP8 && !FMA) {
-            if (a.init_l != nullptr && cs.t0 == 0 && cs.toff > 0) {
+        if constexpr (CAS) {
+            if (cs.t0 == 0 && cs.toff > 0) {
                 // the row's positions before its own blocks were attended by
                 // the shared-prefix kernel: resume from its partial.  Lane
                 // (g8, c4) holds heads 2c4, 2c4+1 of each n-tile at d = 16 mt +

@@ -40,7 +40,11 @@ namespace pkv {
 
 constexpr int kMqRows = 128;      // MMA M: query rows of one unit
 constexpr int kMqTile = 128;      // KV positions per tile (N of Q K^T, K of P V)
-constexpr int kMqThreads = 192;   // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr int kMqSoftmaxWarps = 8;  // two per 32-row quarter: one per 64-column half of S
+constexpr int kMqProducerWarp = 8;   // units, Q and K tiles
+constexpr int kMqMmaWarp = 9;
+constexpr int kMqVProducerWarp = 10; // V tiles
+constexpr int kMqThreads = 352;   // warps 0-7 softmax, 8 K producer, 9 MMA, 10 V producer
 constexpr int kMqKStages = 2;     // K tiles in flight
 constexpr int kMqVStages = 2;     // V tiles in flight
 constexpr float kMqRescaleLog2 = 8.0f;
@@ -87,12 +91,14 @@ struct MqSmem {
     static constexpr int k = q + kTileBytes;
     static constexpr int v = k + kMqKStages * kTileBytes;
     static constexpr int p = v + kMqVStages * kTileBytes;
-    static constexpr int bars = p + kPBytes;
+    static constexpr int xbuf = p + kPBytes;                // [2 parity][2 halves][128 rows] f32
+    static constexpr int bars = xbuf + 2 * 2 * kMqRows * 4;
     // barrier indices
     static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kMqKStages,
                          kVFull = kKEmpty + kMqKStages, kVEmpty = kVFull + kMqVStages, kSFull = kVEmpty + kMqVStages,
                          kSFree = kSFull + 2, kPFull = kSFree + 2, kODone = kPFull + 1, kUnitFull = kODone + 1,
-                         kUnitEmpty = kUnitFull + 2, kDrain = kUnitEmpty + 2, kNumBars = kDrain + 1;
+                         kUnitEmpty = kUnitFull + 2, kDrain = kUnitEmpty + 2, kXch = kDrain + 1,
+                         kNumBars = kXch + 4;
     static constexpr int misc = bars + kNumBars * 8;     // [0..1] unit slots, [2] TMEM base, [3] abort
     static constexpr int prefix = misc + 32;
     static constexpr int bytes(int B) { return prefix + (B + 1) * 4 + 1024; }  // + base re-alignment
@@ -109,10 +115,11 @@ struct MqUnit {
 // Units of source s (0 for sources this kernel does not handle).
 __device__ __forceinline__ int mq_units_of(int s, const MqArgs &a) {
     if (a.mode == kMqPrefix) {
-        const int n = __ldg(a.group_start + s + 1) - __ldg(a.group_start + s);
-        if (n < 1 || __ldg(a.group_len + s) <= 0)
+        const int gs = __ldg(a.group_start + s), ge = __ldg(a.group_start + s + 1);
+        // an invalid or empty group has no reference (its members share nothing)
+        if (gs < 0 || ge > a.B || ge <= gs || __ldg(a.group_len + s) <= 0)
             return 0;
-        return ((n + a.tpb - 1) / a.tpb) * a.Hkv;
+        return ((ge - gs + a.tpb - 1) / a.tpb) * a.Hkv;
     }
     const int q0 = __ldg(a.query_start + s);
     const int n = __ldg(a.query_start + s + 1) - q0;
@@ -178,12 +185,15 @@ __host__ __device__ constexpr uint32_t mq_idesc(bool bf16, int n, bool negate_a,
 }
 
 // Bounded wait that also gives up when another role has aborted; a time-out
-// records the error and raises the abort flag.
+// records the error and raises the abort flag.  The thread sleeps in the
+// wait instruction (woken by the phase's completion) and checks the clock
+// and the abort flag only between sleeps of up to 20 us, so a hand-off costs
+// no polling latency.
 __device__ __forceinline__ bool mq_wait(uint32_t bar, uint32_t parity, const MqArgs &a, volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity))
+    if (mbar_try_wait_hint(bar, parity, 20000u))
         return true;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_hint(bar, parity, 20000u)) {
         if (*abort_flag)
             return false;
         if (global_timer_ns() - t0 > a.wait_limit_ns) {
@@ -207,7 +217,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     constexpr int NH = D / 64;              // 128-byte column halves of a row
     constexpr int kTileBytes = L::kTileBytes;
     constexpr int kHalf = L::kHalf;
-    constexpr uint32_t kTmemCols = 512;     // S0 | S1 | O
+    constexpr uint32_t kTmemCols = 512;     // S0 | S1 | O_0 | O_1 (one O per 64-position half)
     constexpr uint32_t kColO = 256;
     constexpr unsigned FULL = 0xffffffffu;
 
@@ -237,17 +247,19 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(L::kSFull + i), 1);
-            mbar_init(bar(L::kSFree + i), 4);      // one arrival per softmax warp
+            mbar_init(bar(L::kSFree + i), kMqSoftmaxWarps);      // one arrival per softmax warp
             mbar_init(bar(L::kUnitFull + i), 1);
-            mbar_init(bar(L::kUnitEmpty + i), 5);  // the MMA thread + 4 softmax warps
+            mbar_init(bar(L::kUnitEmpty + i), 2 + kMqSoftmaxWarps);  // MMA thread, V producer, softmax warps
         }
-        mbar_init(bar(L::kPFull), 4);
+        mbar_init(bar(L::kPFull), kMqSoftmaxWarps);
+        for (int i = 0; i < 4; ++i)
+            mbar_init(bar(L::kXch + i), 2);  // the two warps of a 32-row quarter
         mbar_init(bar(L::kODone), 1);
         mbar_init(bar(L::kDrain), 1);
         misc[3] = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if ((warp == kMqProducerWarp || warp == kMqVProducerWarp) && lane == 0) {
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
@@ -258,7 +270,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         *reinterpret_cast<uint4 *>(gbase + L::q + h * kHalf + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
-    if (warp == 5) {
+    if (warp == kMqMmaWarp) {
         tmem_alloc(base + L::misc + 8, kTmemCols);
         tmem_relinquish();
     }
@@ -307,105 +319,132 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     const uint32_t tmem = (uint32_t)misc[2];
     const int total = prefix[a.nsrc];
 
-    if (total > 0 && warp == 4) {
-        // ================= producer: unit scheduler + TMA loads =================
+    if (total > 0 && (warp == kMqProducerWarp || warp == kMqVProducerWarp)) {
+        // ================= producers: units + Q + K tiles (warp 8), V tiles (warp 10)
+        // Two warps so that the two tensors' copies are issued in parallel; each
+        // walks the same units.  Per tile, lane l < 8 * NH issues the box of
+        // 16 positions l % 8 in column half l / 8.
+        const bool is_k = warp == kMqProducerWarp;
         int k = 0;
         uint32_t jg = 0;
         int q_issued = -1;                 // last unit whose Q copy was issued
-        int k_last[KS], v_last[VS];        // last use index with copies issued, per stage
-        for (int i = 0; i < KS; ++i)
-            k_last[i] = -1;
-        for (int i = 0; i < VS; ++i)
-            v_last[i] = -1;
+        int t_last[KS > VS ? KS : VS];     // last use index with copies issued, per stage
+        for (int i = 0; i < (KS > VS ? KS : VS); ++i)
+            t_last[i] = -1;
+        const int NS = is_k ? KS : VS;
+        const uint32_t ring = is_k ? sK : sV;
+        const CUtensorMap *tm = is_k ? &tmK : &tmV;
+        const int full0 = is_k ? L::kKFull : L::kVFull, empty0 = is_k ? L::kKEmpty : L::kVEmpty;
         bool ok = true;
         while (ok) {
-            int u = 0;
-            if (lane == 0)
-                u = atomicAdd(a.unit_counter, 1);
-            u = __shfl_sync(FULL, u, 0);
             const int slot = k & 1;
-            ok = __all_sync(FULL, mq_wait(bar(L::kUnitEmpty + slot), ((k >> 1) & 1) ^ 1, a, abort_flag));
-            if (!ok)
-                break;
-            if (lane == 0) {
-                misc[slot] = u < total ? u : -1;
-                mbar_arrive(bar(L::kUnitFull + slot));
+            int u = 0;
+            if (is_k) {
+                if (lane == 0)
+                    u = atomicAdd(a.unit_counter, 1);
+                u = __shfl_sync(FULL, u, 0);
+                ok = __all_sync(FULL, mq_wait(bar(L::kUnitEmpty + slot), ((k >> 1) & 1) ^ 1, a, abort_flag));
+                if (!ok)
+                    break;
+                if (lane == 0) {
+                    misc[slot] = u < total ? u : -1;
+                    mbar_arrive(bar(L::kUnitFull + slot));
+                }
+                if (u >= total)
+                    break;
+            } else {
+                ok = __all_sync(FULL, mq_wait(bar(L::kUnitFull + slot), (k >> 1) & 1, a, abort_flag));
+                if (!ok)
+                    break;
+                u = misc[slot];
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(L::kUnitEmpty + slot));
+                if (u < 0)
+                    break;
             }
-            if (u >= total)
-                break;
             const MqUnit U = mq_unit(u, prefix, a);
-            ok = __all_sync(FULL, mq_wait(bar(L::kQEmpty), (k & 1) ^ 1, a, abort_flag));
-            if (!ok)
-                break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(L::kQFull), (uint32_t)(NH * rows_used * 128));
-                if (!a.inject_no_issue) {
+            if (is_k) {
+                ok = __all_sync(FULL, mq_wait(bar(L::kQEmpty), (k & 1) ^ 1, a, abort_flag));
+                if (!ok)
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(L::kQFull), (uint32_t)(NH * rows_used * 128));
+                    if (!a.inject_no_issue) {
 #pragma unroll
-                    for (int h = 0; h < NH; ++h)
-                        tma_load_3d(sQ + h * kHalf, &tmQ, h * 64, U.kvh * a.G, U.q0 + U.rb * a.tpb, bar(L::kQFull));
-                    q_issued = k;
+                        for (int h = 0; h < NH; ++h)
+                            tma_load_3d(sQ + h * kHalf, &tmQ, h * 64, U.kvh * a.G, U.q0 + U.rb * a.tpb,
+                                        bar(L::kQFull));
+                        q_issued = k;
+                    }
                 }
             }
             const int32_t *trow = a.block_tables + (size_t)U.trow * a.mb;
-            for (int j = 0; j < U.nt && ok; ++j, ++jg) {
-                // lanes 0..7: the pool row of each 16-position box of this tile;
-                // positions past the context (and bad table entries) read zeros
+            const int nblk = (U.ctx + a.bs - 1) / a.bs;
+            // The unit's table entries, 32 at a time: lane i holds entry
+            // cur_base + i; the next 32 are loaded one window ahead so that a
+            // tile never waits for its table entries.
+            auto load_win = [&](int b) { return b + lane < nblk ? __ldg(trow + b + lane) : -1; };
+            int cur_base = 0, cur_val = load_win(0);
+            int nxt_base = 32, nxt_val = load_win(32);
+            // lane l: the pool row of box l % 8 (16 positions) of tile j;
+            // positions past the range (and bad table entries) read zeros
+            auto box_row = [&](int j) {
+                const int b0 = j * kMqTile / a.bs, b1 = min(nblk - 1, (j * kMqTile + kMqTile - 1) / a.bs);
+                if (b0 < cur_base || b1 >= cur_base + 32) {
+                    if (b0 == nxt_base) {
+                        cur_base = nxt_base;
+                        cur_val = nxt_val;
+                    } else {
+                        cur_base = b0;
+                        cur_val = load_win(b0);
+                    }
+                    nxt_base = cur_base + 32;
+                    nxt_val = load_win(nxt_base);
+                }
+                const int pos = j * kMqTile + (lane & 7) * 16;
+                const int blk = __shfl_sync(FULL, cur_val, min(31, max(0, pos / a.bs - cur_base)));
                 int y = a.pool_rows;
-                if (lane < kMqTile / 16) {
-                    const int pos = j * kMqTile + lane * 16;
-                    if (pos < U.ctx) {
-                        const int blk = __ldg(trow + pos / a.bs);
-                        if (blk < 0 || (int64_t)blk >= a.nb)
+                if (pos < U.ctx) {
+                    if (blk < 0 || (int64_t)blk >= a.nb) {
+                        if (is_k && lane < 8)
                             atomicOr(a.err, kErrTable);
-                        else
-                            y = (blk * a.Hkv + U.kvh) * a.bs + pos % a.bs;
+                    } else {
+                        y = (blk * a.Hkv + U.kvh) * a.bs + pos % a.bs;
                     }
                 }
-                const int st = (int)(jg % KS), vt = (int)(jg % VS);
-                ok = __all_sync(FULL, mq_wait(bar(L::kKEmpty + st), ((jg / KS) & 1) ^ 1, a, abort_flag));
+                return y;
+            };
+            for (int j = 0; j < U.nt && ok; ++j) {
+                const uint32_t tg = jg + j;
+                const int y = box_row(j);
+                const int st = (int)(tg % NS);
+                ok = __all_sync(FULL, mq_wait(bar(empty0 + st), ((tg / NS) & 1) ^ 1, a, abort_flag));
                 if (!ok)
                     break;
                 if (lane == 0)
-                    mbar_arrive_expect_tx(bar(L::kKFull + st), kTileBytes);
+                    mbar_arrive_expect_tx(bar(full0 + st), kTileBytes);
                 __syncwarp();
-                if (lane < kMqTile / 16 && !a.inject_no_issue) {
-#pragma unroll
-                    for (int h = 0; h < NH; ++h)
-                        tma_load_2d(sK + st * kTileBytes + h * kHalf + lane * 2048, &tmK, h * 64, y,
-                                    bar(L::kKFull + st));
+                if (lane < 8 * NH && !a.inject_no_issue) {
+                    const int h = lane >> 3;
+                    tma_load_2d(ring + st * kTileBytes + h * kHalf + (lane & 7) * 2048, tm, h * 64, y, bar(full0 + st));
                 }
                 if (!a.inject_no_issue)
-                    k_last[st] = (int)(jg / KS);
-                ok = __all_sync(FULL, mq_wait(bar(L::kVEmpty + vt), ((jg / VS) & 1) ^ 1, a, abort_flag));
-                if (!ok)
-                    break;
-                if (lane == 0)
-                    mbar_arrive_expect_tx(bar(L::kVFull + vt), kTileBytes);
-                __syncwarp();
-                if (lane < kMqTile / 16 && !a.inject_no_issue) {
-#pragma unroll
-                    for (int h = 0; h < NH; ++h)
-                        tma_load_2d(sV + vt * kTileBytes + h * kHalf + lane * 2048, &tmV, h * 64, y,
-                                    bar(L::kVFull + vt));
-                }
-                if (!a.inject_no_issue)
-                    v_last[vt] = (int)(jg / VS);
+                    t_last[st] = (int)(tg / NS);
             }
+            jg += U.nt;
             ++k;
         }
         // copies still in flight land before the CTA may exit (bounded)
         if (lane == 0) {
             if (q_issued >= 0)
                 mbar_wait_bounded(bar(L::kQFull), q_issued & 1, a.wait_limit_ns);
-            for (int i = 0; i < KS; ++i)
-                if (k_last[i] >= 0)
-                    mbar_wait_bounded(bar(L::kKFull + i), k_last[i] & 1, a.wait_limit_ns);
-            for (int i = 0; i < VS; ++i)
-                if (v_last[i] >= 0)
-                    mbar_wait_bounded(bar(L::kVFull + i), v_last[i] & 1, a.wait_limit_ns);
+            for (int i = 0; i < NS; ++i)
+                if (t_last[i] >= 0)
+                    mbar_wait_bounded(bar(full0 + i), t_last[i] & 1, a.wait_limit_ns);
         }
         __syncwarp();
-    } else if (total > 0 && warp == 5) {
+    } else if (total > 0 && warp == kMqMmaWarp) {
         // ================= MMA issuer (one thread) =================
         if (lane == 0) {
             const uint32_t idesc_s = mq_idesc(BF16, kMqTile, a.negate_q != 0, false);
@@ -419,12 +458,18 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                     !mq_wait(bar(L::kVFull + vt), (jp / VS) & 1, a, abort_flag))
                     return false;
                 tc_fence_after();
+                // O_h += P_h V_h for the two 64-position halves h of the tile:
+                // each softmax half keeps its own running max, so each has its
+                // own accumulator (combined once per unit in the epilogue)
 #pragma unroll
-                for (int ks = 0; ks < kMqTile / 16; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(sP + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(sV + vt * kTileBytes + ks * 2048, kHalf, 1024);
-                    tc_mma_ss(tmem + kColO, ad, bd, idesc_o, (first && ks == 0) ? 0u : 1u);
-                }
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int ks = 0; ks < kMqTile / 32; ++ks) {
+                        const uint64_t ad = smem_desc_sw128(sP + h * kHalf + ks * 32, 16, 1024);
+                        const uint64_t bd =
+                            smem_desc_sw128(sV + vt * kTileBytes + h * (kMqTile / 2) * 128 + ks * 2048, kHalf, 1024);
+                        tc_mma_ss(tmem + kColO + h * D, ad, bd, idesc_o, (first && ks == 0) ? 0u : 1u);
+                    }
                 tc_commit(bar(L::kODone));
                 tc_commit(bar(L::kVEmpty + vt));
                 return true;
@@ -476,11 +521,34 @@ __global__ void __launch_bounds__(kMqThreads, 1)
             }
         }
         __syncwarp();
-    } else if (total > 0 && warp < 4) {
-        // ================= softmax + epilogue: thread r owns row r =================
-        const int r = threadIdx.x;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    } else if (total > 0 && warp < kMqSoftmaxWarps) {
+        // ================= softmax + epilogue =================
+        // warp w owns rows 32 (w % 4) .. +31 (its TMEM lane quarter) and
+        // half hc = w / 4 of each tile's 128 positions (64 hc .. 64 hc + 63):
+        // an online softmax of its own over those positions (own running max
+        // and sum) into its own accumulator O_hc.  The two halves of a row
+        // meet once per unit, in the epilogue, through shared memory.
+        const int q4 = warp & 3, hc = warp >> 2;
+        const int r = q4 * 32 + lane;  // row = TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        constexpr int HC = kMqTile / 2;  // positions per warp per tile
+        constexpr int OC = D / 2;        // output columns each warp writes
+        const uint32_t col_o = kColO + hc * D;  // this warp's accumulator
         const int t = r / a.G, hj = r - (r / a.G) * a.G;
+        float *xb = reinterpret_cast<float *>(gbase + L::xbuf);
+        uint32_t xc = 0;  // exchanges done with the partner warp
+        // this warp's value for its rows -> the partner's (bounded wait)
+        auto exchange = [&](float mine, float &theirs) {
+            const int par = (int)(xc & 1);
+            reinterpret_cast<volatile float *>(xb)[(par * 2 + hc) * kMqRows + r] = mine;
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(L::kXch + q4));
+            const bool okx = __all_sync(FULL, mq_wait(bar(L::kXch + q4), xc & 1, a, abort_flag));
+            ++xc;
+            theirs = reinterpret_cast<volatile float *>(xb)[(par * 2 + (hc ^ 1)) * kMqRows + r];
+            return okx;
+        };
         int k = 0;
         uint32_t jg = 0;
         bool ok = true;
@@ -501,37 +569,84 @@ __global__ void __launch_bounds__(kMqThreads, 1)
             int lim = U.lim_max;
             if (valid)
                 lim = a.mode == kMqPrefix ? min(__ldg(a.shared + U.q0 + tok), U.lim_max) : U.ctx - U.n + tok + 1;
-            float m_ref = -INFINITY, l = 0.f;
+            // V rows at positions >= ctx are unwritten (or poisoned) slots:
+            // this thread zeroes column half hc of row r of the tile's V stage
+            // (0 * NaN would leak through P V)
+            auto zero_v_tail = [&](int j) {
+                const int pos0 = j * kMqTile;
+                if (pos0 + kMqTile <= U.ctx)
+                    return true;
+                const int vt = (int)(jg % VS);
+                if (!__all_sync(FULL, mq_wait(bar(L::kVFull + vt), (jg / VS) & 1, a, abort_flag)))
+                    return false;
+                if (pos0 + r >= U.ctx && hc < NH) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t addr = sV + vt * kTileBytes + hc * kHalf + r * 128 + c * 16;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                    }
+                }
+                return true;
+            };
+            // a quarter whose 32 rows are all padding does no softmax work
+            // (its rows of P and O are never read back); its warps still take
+            // part in every hand-off and zero their share of the V rows
+            const bool warp_active = __any_sync(FULL, valid);
+            float m_ref = -INFINITY, l = 0.f;  // this half's running max (log2) and sum
             for (int j = 0; j < U.nt; ++j, ++jg) {
                 ok = __all_sync(FULL, mq_wait(bar(L::kSFull + (jg & 1)), (jg >> 1) & 1, a, abort_flag));
                 if (!ok)
                     break;
                 tc_fence_after();
-                uint32_t sv[kMqTile];
+                if (!warp_active) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar(L::kSFree + (jg & 1)));
+                    if (!(ok = zero_v_tail(j)))
+                        break;
+                    // arrive for this tile only once the previous tile's
+                    // phase is complete (its P V has run): a padding warp must
+                    // not run ahead of the others into the next phase
+                    if (jg > 0) {
+                        ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
+                        if (!ok)
+                            break;
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar(L::kPFull));
+                    continue;
+                }
+                uint32_t sv[HC];
 #pragma unroll
-                for (int c = 0; c < kMqTile / 32; ++c)
-                    tmem_ld32(lane_base + (jg & 1) * kMqTile + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+                for (int c = 0; c < HC / 32; ++c)
+                    tmem_ld32(lane_base + (jg & 1) * kMqTile + hc * HC + c * 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(bar(L::kSFree + (jg & 1)));
-                const int pos0 = j * kMqTile;
-                if (pos0 + kMqTile > lim) {
+                const int pos0 = j * kMqTile + hc * HC;
+                if (pos0 + HC > lim) {
 #pragma unroll
-                    for (int i = 0; i < kMqTile; ++i)
+                    for (int i = 0; i < HC; ++i)
                         if (pos0 + i >= lim)
                             sv[i] = __float_as_uint(-INFINITY);
                 }
-                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+                float mxc[8];
 #pragma unroll
-                for (int i = 0; i < kMqTile; i += 4) {
-                    mx0 = fmaxf(mx0, __uint_as_float(sv[i]));
-                    mx1 = fmaxf(mx1, __uint_as_float(sv[i + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(sv[i + 2]));
-                    mx3 = fmaxf(mx3, __uint_as_float(sv[i + 3]));
-                }
-                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * a.scale_log2;
+                for (int i = 0; i < 8; ++i)
+                    mxc[i] = __uint_as_float(sv[i]);
+#pragma unroll
+                for (int i = 8; i < HC; ++i)
+                    mxc[i & 7] = fmaxf(mxc[i & 7], __uint_as_float(sv[i]));
+                const float mx = fmaxf(fmaxf(fmaxf(mxc[0], mxc[1]), fmaxf(mxc[2], mxc[3])),
+                                       fmaxf(fmaxf(mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]))) *
+                                 a.scale_log2;
                 const float m_new = fmaxf(m_ref, mx);
                 const bool need = m_new > m_ref + kMqRescaleLog2;
                 float alpha = 1.f;
@@ -540,21 +655,21 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                     l *= alpha;
                     m_ref = m_new;
                 }
-                const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;  // a row masked so far: P = 0
-                uint32_t pk[kMqTile / 2];
-                float rs0 = 0.f, rs1 = 0.f;
+                const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;  // a half masked so far: P = 0
+                uint32_t pk[HC / 2];
+                float rsc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < kMqTile / 2; ++i) {
+                for (int i = 0; i < HC / 2; ++i) {
                     const float x0 = fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, neg_m);
                     const float x1 = fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, neg_m);
                     const bool poly = (i & 7) < POLY;
                     const float p0 = poly ? exp2_poly(x0) : exp2f(x0);
                     const float p1 = poly ? exp2_poly(x1) : exp2f(x1);
-                    rs0 += p0;
-                    rs1 += p1;
+                    rsc[(2 * i) & 7] += p0;
+                    rsc[(2 * i + 1) & 7] += p1;
                     pk[i] = pack2<BF16>(p0, p1);
                 }
-                l += rs0 + rs1;
+                l += ((rsc[0] + rsc[1]) + (rsc[2] + rsc[3])) + ((rsc[4] + rsc[5]) + (rsc[6] + rsc[7]));
                 if (j > 0) {
                     // P V of the previous tile is done: P may be overwritten and O rescaled
                     ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
@@ -565,46 +680,28 @@ __global__ void __launch_bounds__(kMqThreads, 1)
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
                             uint32_t o[32];
-                            tmem_ld32(lane_base + kColO + c * 32, o);
+                            tmem_ld32(lane_base + col_o + c * 32, o);
                             tmem_wait_ld();
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
                                 o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                            tmem_st32(lane_base + kColO + c * 32, o);
+                            tmem_st32(lane_base + col_o + c * 32, o);
                         }
                         tmem_wait_st();
                     }
                 }
-                // P -> shared memory, K-major 128-byte swizzle: positions
-                // 64h .. 64h+63 of row r at sP + h*kHalf + r*128, 16-byte chunk c
-                // at (c ^ (r % 8)) * 16
+                // P_hc -> shared memory, K-major 128-byte swizzle: positions
+                // 64 hc .. 64 hc + 63 of row r at sP + hc*kHalf + r*128, 16-byte
+                // chunk c at (c ^ (r % 8)) * 16
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t addr = sP + h * kHalf + r * 128 + ((c ^ (r & 7)) << 4);
-                        const int b = h * 32 + c * 4;
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[b]),
-                                     "r"(pk[b + 1]), "r"(pk[b + 2]), "r"(pk[b + 3])
-                                     : "memory");
-                    }
-                if (pos0 + kMqTile > U.ctx) {
-                    // V rows at positions >= ctx are unwritten (or poisoned) slots
-                    const int vt = (int)(jg % VS);
-                    ok = __all_sync(FULL, mq_wait(bar(L::kVFull + vt), (jg / VS) & 1, a, abort_flag));
-                    if (!ok)
-                        break;
-                    if (pos0 + r >= U.ctx) {
-#pragma unroll
-                        for (int h = 0; h < NH; ++h)
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const uint32_t addr = sV + vt * kTileBytes + h * kHalf + r * 128 + c * 16;
-                                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
-                                             : "memory");
-                            }
-                    }
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t addr = sP + hc * kHalf + r * 128 + ((c ^ (r & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c * 4]),
+                                 "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
+                                 : "memory");
                 }
+                if (!(ok = zero_v_tail(j)))
+                    break;
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -613,40 +710,60 @@ __global__ void __launch_bounds__(kMqThreads, 1)
             }
             if (!ok)
                 break;
-            // ---- epilogue: O / l of every valid row
+            // ---- epilogue: the two halves of each row combined,
+            //   M = max(m_0, m_1), f_h = 2^(m_h - M) (0 for an empty half),
+            //   out = (f_0 O_0 + f_1 O_1) / (f_0 l_0 + f_1 l_1);
+            // this warp writes output columns OC hc .. OC hc + OC - 1
+            if (!warp_active) {
+                ++k;
+                continue;
+            }
             ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
             if (!ok)
                 break;
+            float m_o, l_o;
+            if (!(ok = exchange(m_ref, m_o)) || !(ok = exchange(l, l_o)))
+                break;
+            const float m0 = hc == 0 ? m_ref : m_o, m1 = hc == 0 ? m_o : m_ref;
+            const float l0 = hc == 0 ? l : l_o, l1 = hc == 0 ? l_o : l;
+            const float M = fmaxf(m0, m1);
+            const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+            const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+            const float l_row = f0 * l0 + f1 * l1;
             tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
             const size_t orow_idx = (size_t)(U.q0 + (valid ? tok : 0)) * a.Hq + U.kvh * a.G + hj;
-            uint16_t *orow = a.out + orow_idx * D;
-            if (a.mode == kMqPrefix && valid) {
-                a.part_m[orow_idx] = m_ref;
-                a.part_l[orow_idx] = l;
+            uint16_t *orow = a.out + orow_idx * D + hc * OC;
+            if (a.mode == kMqPrefix && valid && hc == 0) {
+                a.part_m[orow_idx] = M;
+                a.part_l[orow_idx] = l_row;
             }
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + kColO + c * 32, o);
+            for (int c = 0; c < OC / 32; ++c) {
+                uint32_t o0[32], o1[32];
+                tmem_ld32(lane_base + kColO + hc * OC + c * 32, o0);
+                tmem_ld32(lane_base + kColO + D + hc * OC + c * 32, o1);
                 tmem_wait_ld();
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = f0 * __uint_as_float(o0[i]) + f1 * __uint_as_float(o1[i]);
                 if (a.mode == kMqPrefix) {
-                    // unnormalized fp32 partial, relative to 2^m_ref
+                    // unnormalized fp32 partial, relative to 2^M
                     if (valid) {
-                        float4 *dst = reinterpret_cast<float4 *>(a.part_o + orow_idx * D + c * 32);
+                        float4 *dst = reinterpret_cast<float4 *>(a.part_o + orow_idx * D + hc * OC + c * 32);
 #pragma unroll
                         for (int v4 = 0; v4 < 8; ++v4)
-                            dst[v4] = make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
-                                                  __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
+                            dst[v4] = make_float4(v[4 * v4], v[4 * v4 + 1], v[4 * v4 + 2], v[4 * v4 + 3]);
                     }
                 } else if (valid) {
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
                         uint4 w;
-                        w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * inv, __uint_as_float(o[v4 * 8 + 1]) * inv);
-                        w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * inv, __uint_as_float(o[v4 * 8 + 3]) * inv);
-                        w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * inv, __uint_as_float(o[v4 * 8 + 5]) * inv);
-                        w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * inv, __uint_as_float(o[v4 * 8 + 7]) * inv);
+                        w.x = pack2<BF16>(v[v4 * 8 + 0] * inv, v[v4 * 8 + 1] * inv);
+                        w.y = pack2<BF16>(v[v4 * 8 + 2] * inv, v[v4 * 8 + 3] * inv);
+                        w.z = pack2<BF16>(v[v4 * 8 + 4] * inv, v[v4 * 8 + 5] * inv);
+                        w.w = pack2<BF16>(v[v4 * 8 + 6] * inv, v[v4 * 8 + 7] * inv);
                         *reinterpret_cast<uint4 *>(orow + c * 32 + v4 * 8) = w;
                     }
                 }
@@ -659,7 +776,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5)
+    if (warp == kMqMmaWarp)
         tmem_dealloc(tmem, kTmemCols);
 }
 
@@ -667,93 +784,124 @@ __global__ void __launch_bounds__(kMqThreads, 1)
 
 namespace pkv {
 
-// Preparation of a shared-prefix decode step (one CTA).  For every sequence
-// the defaults (no shared prefix: whole context left to the decode kernel);
-// then one warp per sharing group: the reference member (the first with the
-// largest claimed shared length), each member's effective shared length --
-// its claim, capped so that its last position stays in its own blocks, and
-// cut at the first table entry that differs from the reference's -- the
-// group's longest, and each member's remaining length and table offset for
-// the decode kernel.  A claim that does not hold only shrinks the shared
-// part, so the result stays exact.
-__global__ void __launch_bounds__(1024) cascade_prep_kernel(
+// Preparation of a shared-prefix decode step: one warp per sequence.  The
+// sequence's group (binary search of group_start, staged in shared memory);
+// the group's reference (the first member with the largest claim, each
+// claim in whole blocks and cut so that the member's last position -- this
+// step's token -- stays in its own blocks); the sequence's effective shared
+// length (its claim, cut at the first table entry that differs from the
+// reference's: 32 entries compared per round); its remaining (suffix)
+// length and table offset for the decode kernel; and (every member, the same
+// values) the group's reference row and KV range.  A claim that does not hold
+// only shrinks the shared part, so the result stays exact.  An invalid
+// group_start shares nothing and is reported.
+__global__ void __launch_bounds__(256) cascade_prep_kernel(
     const int32_t *__restrict__ group_start, int NG, const int32_t *__restrict__ claimed,
     const int32_t *__restrict__ context_lens, const int32_t *__restrict__ block_tables, int64_t mb, int bs,
     int B, int32_t *group_ref, int32_t *group_len, int32_t *shared, int32_t *suffix_len, int32_t *table_off,
     int *mq_counter, unsigned *err) {
     constexpr unsigned FULL = 0xffffffffu;
+    extern __shared__ int gs_s[];  // group_start[0 .. NG]
     griddep_wait();
-    if (threadIdx.x == 0)
+    griddep_launch_dependents();
+    if (blockIdx.x == 0 && threadIdx.x == 0)
         *mq_counter = 0;
+    for (int i = threadIdx.x; i <= NG; i += blockDim.x)
+        gs_s[i] = __ldg(group_start + i);
+    __syncthreads();
+    // group_start must run from 0 to B without decreasing; otherwise nothing
+    // is shared (every group length 0) and the fault is reported
+    int bad = 0;
+    for (int i = threadIdx.x; i <= NG; i += blockDim.x)
+        bad |= (i == 0 && gs_s[0] != 0) || (i == NG && gs_s[NG] != B) || (i < NG && gs_s[i + 1] < gs_s[i]);
+    if (__syncthreads_or(bad)) {
+        if (threadIdx.x == 0)
+            atomicOr(err, kErrContext);
+        for (int i = threadIdx.x; i < NG; i += blockDim.x)
+            group_len[i] = 0;
+        for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < B; s += gridDim.x * blockDim.x) {
+            const int c = __ldg(context_lens + s);
+            const int64_t cap = mb * bs;
+            shared[s] = 0;
+            suffix_len[s] = c < 0 ? 0 : ((int64_t)c > cap ? (int)cap : c);
+            table_off[s] = 0;
+        }
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (m >= B)
+        return;
     const int64_t cap = mb * bs;
     auto ctx_of = [&](int s) {
         const int c = __ldg(context_lens + s);
-        if (c < 0 || (int64_t)c > cap) {
-            atomicOr(err, kErrContext);
-            return c < 0 ? 0 : (int)cap;
-        }
-        return c;
+        return c < 0 ? 0 : ((int64_t)c > cap ? (int)cap : c);
     };
-    for (int s = threadIdx.x; s < B; s += blockDim.x) {
-        shared[s] = 0;
-        suffix_len[s] = ctx_of(s);
-        table_off[s] = 0;
+    // claim in whole blocks, the sequence's last position kept private
+    auto claim_blocks = [&](int s) {
+        const int c = ctx_of(s);
+        const int cl = __ldg(claimed + s);
+        return (c < 1 || cl <= 0) ? 0 : min(cl, c - 1) / bs;
+    };
+    const int ctx = ctx_of(m);
+    {
+        const int c = __ldg(context_lens + m);
+        if (lane == 0 && (c < 0 || (int64_t)c > cap))
+            atomicOr(err, kErrContext);
     }
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warps = blockDim.x >> 5;
-    for (int g = threadIdx.x >> 5; g < NG; g += warps) {
-        int gs = __ldg(group_start + g), ge = __ldg(group_start + g + 1);
-        if (gs < 0 || ge > B || ge < gs) {
-            if (lane == 0)
-                atomicOr(err, kErrContext);
-            gs = ge = 0;
-        }
-        // claims in whole blocks, the sequence's last position kept private
-        auto claim_blocks = [&](int m) {
-            const int c = ctx_of(m);
-            const int cl = __ldg(claimed + m);
-            if (c < 1 || cl <= 0)
-                return 0;
-            return min(cl, c - 1) / bs;
-        };
-        int best = -1, best_c = -1;
-        for (int m = gs + lane; m < ge; m += 32) {
-            const int c = claim_blocks(m);
-            if (c > best_c) {
-                best_c = c;
-                best = m;
+    int e = 0;  // shared blocks of m
+    // the group holding m: the last g with group_start[g] <= m
+    int lo = 0, hi = NG + 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (gs_s[mid] <= m)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    const int g = lo - 1;  // valid: group_start runs from 0 to B
+    {
+        const int gs = gs_s[g], ge = gs_s[g + 1];
+        {
+            int best = -1, best_c = -1;
+            for (int q = gs + lane; q < ge; q += 32) {
+                const int c = claim_blocks(q);
+                if (c > best_c) {
+                    best_c = c;
+                    best = q;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const int oc = __shfl_xor_sync(FULL, best_c, o), om = __shfl_xor_sync(FULL, best, o);
+                if (oc > best_c || (oc == best_c && om >= 0 && (best < 0 || om < best))) {
+                    best_c = oc;
+                    best = om;
+                }
+            }
+            const int ref = best;
+            const int cb = min(claim_blocks(m), best_c);
+            const int32_t *tm = block_tables + (size_t)m * mb, *tr = block_tables + (size_t)ref * mb;
+            while (e < cb) {
+                const int i = e + lane;
+                const bool eq = i >= cb || __ldg(tm + i) == __ldg(tr + i);
+                const unsigned diff = __ballot_sync(FULL, !eq);
+                if (diff) {
+                    e += __ffs(diff) - 1;
+                    break;
+                }
+                e = min(cb, e + 32);
+            }
+            if (lane == 0) {  // every member writes the same values
+                group_ref[g] = ref;
+                group_len[g] = best_c * bs;
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const int oc = __shfl_xor_sync(FULL, best_c, o), om = __shfl_xor_sync(FULL, best, o);
-            if (oc > best_c || (oc == best_c && om >= 0 && (best < 0 || om < best))) {
-                best_c = oc;
-                best = om;
-            }
-        }
-        const int ref = best < 0 ? gs : best;
-        const int ref_blocks = best_c < 0 ? 0 : best_c;
-        const int32_t *tr = block_tables + (size_t)ref * mb;
-        int glen = 0;
-        for (int m = gs + lane; m < ge; m += 32) {
-            const int cb = min(claim_blocks(m), ref_blocks);
-            const int32_t *tm = block_tables + (size_t)m * mb;
-            int e = 0;
-            while (e < cb && __ldg(tm + e) == __ldg(tr + e))
-                ++e;
-            shared[m] = e * bs;
-            suffix_len[m] = ctx_of(m) - e * bs;
-            table_off[m] = e;
-            glen = max(glen, e * bs);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            glen = max(glen, __shfl_xor_sync(FULL, glen, o));
-        if (lane == 0) {
-            group_ref[g] = ref;
-            group_len[g] = glen;
-        }
+    }
+    if (lane == 0) {
+        shared[m] = e * bs;
+        suffix_len[m] = ctx - e * bs;
+        table_off[m] = e;
     }
 }
 

@@ -193,7 +193,23 @@ using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const Decode
 // NT = number of 8-head MMA column tiles per unit: 1 for G <= 8, else 2.
 // bf16: q / out dtype; fp8: E4M3 pools; fma: the CUDA-core variant (16-bit
 // pools, 8 heads per unit), kept to compare against the MMA kernel.
-DecodeKernel pick_decode(int D, bool bf16, int nt, bool fp8 = false, bool fma = false) {
+DecodeKernel pick_decode(int D, bool bf16, int nt, bool fp8 = false, bool fma = false, bool cas = false) {
+    if (cas) {
+        if (fp8 || fma)
+            return nullptr;
+#define PKV_PICK_CAS(DD, BB, NN) \
+    if (D == DD && bf16 == BB && nt == NN) return paged_decode_kernel<DD, BB, NN, false, false, true>;
+        PKV_PICK_CAS(64, false, 1)
+        PKV_PICK_CAS(64, false, 2)
+        PKV_PICK_CAS(64, true, 1)
+        PKV_PICK_CAS(64, true, 2)
+        PKV_PICK_CAS(128, false, 1)
+        PKV_PICK_CAS(128, false, 2)
+        PKV_PICK_CAS(128, true, 1)
+        PKV_PICK_CAS(128, true, 2)
+#undef PKV_PICK_CAS
+        return nullptr;
+    }
     if (fma) {
         if (fp8 || nt != 1)
             return nullptr;
@@ -462,12 +478,27 @@ pkv_status mq_launch(MqArgs a, const void *q, int64_t nz, const pkv_cache &kc, c
     smem = std::max(smem, kMaxSmemPerCta / 2 + 1024);
     if (smem > kMaxSmemPerCta)
         return PKV_ERR_INVALID;
-    if (!cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta)))
-        return PKV_ERR_CUDA;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return PKV_ERR_CUDA;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    {
+        // shared-memory ceiling and SM count, once per (device, kernel)
+        static std::mutex mu;
+        static std::vector<std::tuple<int, const void *, int>> done;
+        std::lock_guard<std::mutex> lock(mu);
+        bool found = false;
+        for (auto &e : done)
+            if (std::get<0>(e) == dev && std::get<1>(e) == (const void *)k) {
+                sms = std::get<2>(e);
+                found = true;
+            }
+        if (!found) {
+            if (!cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta)))
+                return PKV_ERR_CUDA;
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            done.emplace_back(dev, (const void *)k, sms);
+        }
+    }
     if (!cuda_ok(launch_dependent(k, dim3(sms), dim3(kMqThreads), smem, (cudaStream_t)stream, tmQ, tmK, tmV, a)))
         return PKV_ERR_CUDA;
     return PKV_OK;
@@ -686,7 +717,24 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.k_scales = k_cache.scales;
     a.v_scales = v_cache.scales;
 
-    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8, p.fma);
+    DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8, p.fma, cas != nullptr);
+    if (!k)
+        return PKV_ERR_INVALID;
+    if (cas) {
+        // the cascade instantiation shares the plan of the plain kernel; give
+        // it the same shared-memory ceiling once per device
+        static std::mutex mu;
+        static std::vector<std::pair<int, DecodeKernel>> done;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        std::lock_guard<std::mutex> lock(mu);
+        if (std::find(done.begin(), done.end(), std::make_pair(dev, k)) == done.end()) {
+            if (!cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta)))
+                return PKV_ERR_CUDA;
+            done.emplace_back(dev, k);
+        }
+    }
     if (!cuda_ok(launch_dependent(k, dim3(p.ctas), dim3(p.warps * 32), p.smem, (cudaStream_t)stream, tmK,
                                   tmV, a)))
         return PKV_ERR_CUDA;
@@ -926,7 +974,7 @@ pkv_status pkv_append_decode_attention_shared_prefix(
     float *po = reinterpret_cast<float *>(ws + wl.o);
     float *pm = reinterpret_cast<float *>(ws + wl.m);
     float *pl = reinterpret_cast<float *>(ws + wl.l);
-    cascade_prep_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(
+    cascade_prep_kernel<<<(unsigned)((num_seqs + 7) / 8), 256, (size_t)(num_groups + 1) * 4, (cudaStream_t)stream>>>(
         group_start, (int)num_groups, shared_lens, context_lens, block_tables, max_blocks_per_seq,
         (int)k_cache.block_size, (int)num_seqs, g_ref, g_len, shared, suffix, toff, counter, err);
     if (!cuda_ok(cudaGetLastError()))
