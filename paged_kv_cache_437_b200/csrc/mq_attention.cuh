@@ -637,15 +637,15 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                         if (pos0 + i >= lim)
                             sv[i] = __float_as_uint(-INFINITY);
                 }
+                // row max: eight independent chains of three-input maxima
                 float mxc[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    mxc[i] = __uint_as_float(sv[i]);
+                    mxc[i] = fmaxf(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
 #pragma unroll
-                for (int i = 8; i < HC; ++i)
-                    mxc[i & 7] = fmaxf(mxc[i & 7], __uint_as_float(sv[i]));
-                const float mx = fmaxf(fmaxf(fmaxf(mxc[0], mxc[1]), fmaxf(mxc[2], mxc[3])),
-                                       fmaxf(fmaxf(mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]))) *
+                for (int i = 16; i < HC; i += 2)
+                    mxc[(i >> 1) & 7] = fmax3(mxc[(i >> 1) & 7], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+                const float mx = fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], fmax3(mxc[4], mxc[5], mxc[6]), mxc[7])) *
                                  a.scale_log2;
                 const float m_new = fmaxf(m_ref, mx);
                 const bool need = m_new > m_ref + kMqRescaleLog2;
@@ -656,20 +656,24 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                     m_ref = m_new;
                 }
                 const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;  // a half masked so far: P = 0
+                // exponent arguments and row sums on packed fp32 pairs (one
+                // instruction per two elements)
                 uint32_t pk[HC / 2];
-                float rsc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                const uint64_t c2 = f32x2_pack(a.scale_log2, a.scale_log2), nm2 = f32x2_pack(neg_m, neg_m);
+                uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int i = 0; i < HC / 2; ++i) {
-                    const float x0 = fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, neg_m);
-                    const float x1 = fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, neg_m);
+                    const float2 x = f32x2_unpack(
+                        f32x2_fma(f32x2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nm2));
                     const bool poly = (i & 7) < POLY;
-                    const float p0 = poly ? exp2_poly(x0) : exp2f(x0);
-                    const float p1 = poly ? exp2_poly(x1) : exp2f(x1);
-                    rsc[(2 * i) & 7] += p0;
-                    rsc[(2 * i + 1) & 7] += p1;
+                    const float p0 = poly ? exp2_poly(x.x) : exp2f(x.x);
+                    const float p1 = poly ? exp2_poly(x.y) : exp2f(x.y);
+                    rs2[i & 3] = f32x2_add(rs2[i & 3], f32x2_pack(p0, p1));
                     pk[i] = pack2<BF16>(p0, p1);
                 }
-                l += ((rsc[0] + rsc[1]) + (rsc[2] + rsc[3])) + ((rsc[4] + rsc[5]) + (rsc[6] + rsc[7]));
+                const float2 r01 = f32x2_unpack(f32x2_add(rs2[0], rs2[1]));
+                const float2 r23 = f32x2_unpack(f32x2_add(rs2[2], rs2[3]));
+                l += (r01.x + r01.y) + (r23.x + r23.y);
                 if (j > 0) {
                     // P V of the previous tile is done: P may be overwritten and O rescaled
                     ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
