@@ -52,8 +52,10 @@ if ROOT not in sys.path:
 METRIC = "paged decode attention: achieved HBM GB/s (% of B200 peak); decode tokens/s/layer"
 DEFAULT_WORKLOAD = "llama13b"
 PROFILE_DIR = os.path.join(ROOT, "profiles")
+# the sources the decode kernel's profiled traffic depends on (its code, the
+# instruction wrappers and the host plan that sizes its launch)
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_437_b200", "csrc", f)
-                  for f in ("decode.cuh", "mq_attention.cuh", "ptx.cuh", "pkv_cuda.cu")]
+                  for f in ("decode.cuh", "ptx.cuh", "pkv_cuda.cu")]
 
 
 # ------------------------------------------------------------------ bytes
@@ -243,9 +245,10 @@ def run_gpu(args, rank, world, local):
     # built up to ctx - 1 tokens (prefix blocks shared through fork).
     alloc = pkv.BlockAllocator(w.num_blocks, sp.block_size)
     slots_np, alloc_us, groups = allocator_slots(pkv, alloc, w)
-    # a workload whose sequences share prefix blocks runs its step through the
-    # shared-prefix call (each group's prefix read once); --no-cascade: plain
-    cascade = groups is not None and not args.no_cascade and not args.unfused
+    # --cascade: a workload whose sequences share prefix blocks runs its step
+    # through the shared-prefix call (each group's prefix read once) instead of
+    # the plain decode step
+    cascade = groups is not None and args.cascade and not args.unfused
 
     q = dev(w.q)
     kc, vc = dev(w.k_cache), dev(w.v_cache)
@@ -296,8 +299,8 @@ def run_gpu(args, rank, world, local):
                       vdesc, tables.data_ptr(), tables.shape[1], lens.data_ptr(), gstart.data_ptr(), ngroups,
                       claims.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, sptr)
 
-    def make_step(q, kn, vn, slots, tables, lens, gstart=None, claims=None):
-        """The step's raw C ABI calls on these device inputs."""
+    def make_step(q, kn, vn, slots, tables, lens, gstart=None, claims=None, out=out):
+        """The step's raw C ABI calls on these device inputs (and output)."""
         a_args = (kn.data_ptr(), vn.data_ptr(), slots.data_ptr(), slots.numel(), kdesc, vdesc, sptr)
         d_args = (q.data_ptr(), q.shape[0], q.shape[1], kdesc, vdesc, tables.data_ptr(), tables.shape[1],
                   lens.data_ptr(), ctypes.c_float(w.scale), out.data_ptr(), ws_ptr, ws_bytes, part, sptr)
@@ -493,7 +496,9 @@ def measure_e2e(args, make_step, stream, inputs, out):
     memory: q, the new K/V, slots, tables and lengths (and the sharing groups,
     when the step uses them) packed into one pinned staging buffer and sent
     with one host-to-device copy, the kernels, and one device-to-host copy of
-    the output, all inside the timed region."""
+    the output, all inside the timed region.  As a serving loop would, the
+    copies run on their own stream, double-buffered: step k+1's inputs go up
+    and step k-1's output comes down while step k computes."""
     import torch
 
     offs, off = [], 0
@@ -502,31 +507,57 @@ def measure_e2e(args, make_step, stream, inputs, out):
         offs.append(off)
         off += t.numel() * t.element_size()
     h_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
-    d_buf = torch.empty(off, dtype=torch.uint8, device="cuda")
-    views = []
     for t, o in zip(inputs, offs):
         n = t.numel() * t.element_size()
         h_buf[o:o + n].copy_(t.reshape(-1).view(torch.uint8).cpu())
-        views.append(d_buf[o:o + n].view(t.dtype).view(t.shape))
-    step = make_step(*views)
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_buf = [torch.empty(off, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    d_out = [torch.empty_like(out) for _ in range(2)]
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    steps = []
+    for b in range(2):
+        views = [d_buf[b][o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                 for t, o in zip(inputs, offs)]
+        steps.append(make_step(*views, out=d_out[b]))
     h2d = sum(t.numel() * t.element_size() for t in inputs)
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_out[0].numel() * h_out[0].element_size()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()  # uploads never queue behind downloads
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev(), ev()]
+    computed = [ev(), ev()]
+    out_done = [ev(), ev()]
+    started = [False, False]
 
-    def e2e_step():
-        d_buf.copy_(h_buf, non_blocking=True)
-        step()
-        h_out.copy_(out, non_blocking=True)
+    def run(n):
+        for k in range(n):
+            b = k & 1
+            with torch.cuda.stream(up):
+                if started[b]:
+                    up.wait_event(computed[b])                # step k-2 has read d_buf[b]
+                d_buf[b].copy_(h_buf, non_blocking=True)
+                in_ready[b].record(up)
+            stream.wait_event(in_ready[b])
+            if started[b]:
+                stream.wait_event(out_done[b])                # step k-2's output is down
+            steps[b]()
+            computed[b].record(stream)
+            started[b] = True
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                h_out[b].copy_(d_out[b], non_blocking=True)
+                out_done[b].record(down)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    run(max(2, args.warmup))
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(up)
+    stream.wait_event(e0)
+    down.wait_event(e0)
+    run(args.steps)
+    # the region ends when the last output is on the host
+    down.wait_stream(stream)
+    down.wait_stream(up)
+    e1.record(down)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1))
     barrier()
@@ -935,8 +966,8 @@ def parse_args(argv=None):
                     help="step = pkv_append + pkv_decode_attention (default: pkv_append_decode_attention)")
     ap.add_argument("--chunks-only", action="store_true",
                     help="--row prefill: time only the two prefill chunks (a small case for profiling)")
-    ap.add_argument("--no-cascade", action="store_true",
-                    help="workloads with shared prefixes: plain decode step instead of the shared-prefix call")
+    ap.add_argument("--cascade", action="store_true",
+                    help="workloads with shared prefixes: the shared-prefix call instead of the plain decode step")
     ap.add_argument("--seqs", type=int, default=None,
                     help="run the workload with its first N sequences only (small profiling cases)")
     args = ap.parse_args(argv)
@@ -1017,10 +1048,11 @@ def main(argv=None):
             import workloads
 
             subs = {}
-            for name in EXTRA_WORKLOADS:
+            for name in EXTRA_WORKLOADS + ("cb_mixed_shared_prefix",):
                 a2 = copy.copy(args)
-                a2.workload = name
-                a2.partition = workloads.CONFIGS[name].partition_tokens or 0
+                a2.workload = "cb_mixed" if name == "cb_mixed_shared_prefix" else name
+                a2.cascade = name == "cb_mixed_shared_prefix"
+                a2.partition = workloads.CONFIGS[a2.workload].partition_tokens or 0
                 a2.no_cpu_baseline = True
                 subs[name] = workload_summary(run_gpu(a2, rank, world, local))
                 torch.cuda.empty_cache()

@@ -71,6 +71,10 @@ struct DecodeArgs {
     float *part_m;
     float *part_l;
     int32_t *prefix_out;           // balanced: tile prefix for the merge kernel
+    // balanced: one counter per (sequence, head group), zero at launch; the
+    // warp that finishes the last piece of a split row merges it (no merge
+    // kernel).  Null: the merge kernel does it.
+    int *fold_cnt;
     int total_warps;
     int stages;
     unsigned *err;
@@ -307,6 +311,188 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
 
 __device__ __forceinline__ void sts_f4(uint32_t addr, float x, float y, float z, float w) {
     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(x), "f"(y), "f"(z), "f"(w) : "memory");
+}
+
+// ------------------------------------------------------------- merging split rows
+// (used by the merge kernel and by the decode kernel's last piece of a row)
+
+struct MergeArgs {
+    uint16_t *out;
+    const int32_t *context_lens;
+    const int32_t *prefix;   // balanced: tile prefix written by the decode kernel
+    const float *part_o, *part_m, *part_l;
+    int64_t mb;
+    int B, Hq, G, n_hg, npairs, bs;
+    int hpu;                 // query heads per decode unit (8 or 16)
+    int mode, part_tiles, S, total_warps;
+};
+// Balanced mode: prefix[B + 1] holds an upper bound on the pieces per row;
+// partition mode: S is the bound.
+
+constexpr int kMergeThreads = 128;
+constexpr int kMergeWideThreads = 512;  // one row per CTA, many pieces per row
+
+template <int NTH>
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
+    constexpr unsigned FULL = 0xffffffffu;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float x = __shfl_xor_sync(FULL, v, o);
+        v = is_max ? fmaxf(v, x) : v + x;
+    }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0)
+        red[warp] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int w = 1; w < NTH / 32; ++w)
+        r = is_max ? fmaxf(r, red[w]) : r + red[w];
+    __syncthreads();
+    return r;
+}
+
+// Where the pieces of one query head's split context are.
+struct MergeRow {
+    int seq, h, g;
+    long long count;   // pieces; <= 1 means nothing to merge
+    long long first;   // balanced: first warp
+    long long a0, T;   // balanced: flattened start of the pair, total tiles
+};
+
+__device__ __forceinline__ MergeRow merge_row(const MergeArgs &a, long long row) {
+    MergeRow r;
+    r.seq = (int)(row / a.Hq);
+    r.h = (int)(row - (long long)r.seq * a.Hq);
+    const int kvh = r.h / a.G;
+    const int hl = r.h - kvh * a.G;
+    const int hg = hl / a.hpu;
+    r.g = hl - hg * a.hpu;
+    const int pair = kvh * a.n_hg + hg;
+    r.first = 0;
+    r.a0 = 0;
+    r.T = 1;
+    if (a.mode == kModePartition) {
+        int c = a.context_lens[r.seq];
+        const int64_t cap = a.mb * a.bs;
+        c = c < 0 ? 0 : (c > cap ? (int)cap : c);
+        const int nt = (c + kTileTokens - 1) / kTileTokens;
+        r.count = (nt + a.part_tiles - 1) / a.part_tiles;  // <= 1: written by the decode kernel
+    } else {
+        const int nt = a.prefix[r.seq + 1] - a.prefix[r.seq];
+        r.count = 0;
+        if (nt > 0) {
+            r.T = (long long)a.prefix[a.B] * a.npairs;
+            r.a0 = (long long)a.prefix[r.seq] * a.npairs + (long long)pair * nt;
+            const long long W = a.total_warps;
+            r.first = ((r.a0 + 1) * W + r.T - 1) / r.T - 1;                 // warp holding a0
+            const long long last = ((r.a0 + nt) * W + r.T - 1) / r.T - 1;  // warp holding a0+nt-1
+            r.count = last - r.first + 1;  // 1: the pair sat in one warp, already final
+        }
+    }
+    return r;
+}
+
+// Partial row of piece k, or -1 (a warp whose range is empty).
+__device__ __forceinline__ long long merge_piece(const MergeArgs &a, const MergeRow &r, long long k) {
+    if (a.mode == kModePartition)
+        return ((long long)r.seq * a.Hq + r.h) * a.S + k;
+    const long long w = r.first + k;
+    if (r.T >= a.total_warps) {
+        // no warp has an empty range: the first piece is the first warp's
+        // last segment (slot 1), every later piece its warp's first (slot 0)
+        return (2 * w + (k == 0 ? 1 : 0)) * kMaxRows + r.g;
+    }
+    const long long lo = w * r.T / a.total_warps;
+    const long long hi = (w + 1) * r.T / a.total_warps;
+    if (lo >= hi)
+        return -1;
+    return (2 * w + (r.a0 < lo ? 0 : 1)) * kMaxRows + r.g;
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ void store_row(const MergeArgs &a, const MergeRow &r, int c, const float *v,
+                                          int n) {
+    uint32_t *dst = reinterpret_cast<uint32_t *>(a.out + ((size_t)r.seq * a.Hq + r.h) * D + c);
+    for (int i = 0; i < n / 2; ++i)
+        dst[i] = pack2<BF16>(v[2 * i], v[2 * i + 1]);
+}
+
+constexpr int kWarpPieces = 64;  // rows with at most this many pieces: one warp each
+
+// One warp merges one row, kWarpBatch pieces at a time (rescaled online
+// across batches).  A piece's output row does not depend on its weight, so
+// each batch issues every load at once: lane j < kWarpBatch fetches piece
+// j's (m, l), every lane its D/32 columns of all the batch's outputs; the
+// reductions are shuffles.  One memory round trip per batch.
+constexpr int kWarpBatch = 16;
+
+template <int D, bool BF16, int kWarpBatch = kWarpBatch>
+__device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRow &r) {
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int VEC = D / 32;
+    const int lane = threadIdx.x & 31;
+    float M = -INFINITY, L = 0.f;
+    float acc[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i)
+        acc[i] = 0.f;
+    for (long long k0 = 0; k0 < r.count; k0 += kWarpBatch) {
+        const long long kl = k0 + lane;
+        const long long rl = (lane < kWarpBatch && kl < r.count) ? merge_piece(a, r, kl) : -1;
+        const float ml = rl >= 0 ? a.part_m[rl] : -INFINITY;
+        const float ll = rl >= 0 ? a.part_l[rl] : 0.f;
+        float v[kWarpBatch][VEC];
+#pragma unroll
+        for (int j = 0; j < kWarpBatch; ++j) {
+            const long long rr = __shfl_sync(FULL, rl, j);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i)
+                v[j][i] = 0.f;
+            if (rr >= 0) {  // an empty piece (-1) has no row
+                const float *p = a.part_o + rr * D + lane * VEC;
+                if constexpr (VEC == 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(p);
+                    v[j][0] = x.x;
+                    v[j][1 % VEC] = x.y;
+                    v[j][2 % VEC] = x.z;
+                    v[j][3 % VEC] = x.w;
+                } else {
+                    const float2 x = *reinterpret_cast<const float2 *>(p);
+                    v[j][0] = x.x;
+                    v[j][1 % VEC] = x.y;
+                }
+            }
+        }
+        float cm = ml;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
+        const float mnew = fmaxf(M, cm);
+        const float rescale = M == -INFINITY ? 0.f : exp2f(M - mnew);
+        const float w = ml == -INFINITY ? 0.f : exp2f(ml - mnew);
+        float lsum = w * ll;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            lsum += __shfl_xor_sync(FULL, lsum, o);
+        L = L * rescale + lsum;
+        M = mnew;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i)
+            acc[i] *= rescale;
+#pragma unroll
+        for (int j = 0; j < kWarpBatch; ++j) {
+            const float wj = __shfl_sync(FULL, w, j);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i)
+                acc[i] = wj != 0.f ? fmaf(wj, v[j][i], acc[i]) : acc[i];
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i)
+        acc[i] *= inv;
+    store_row<D, BF16>(a, r, lane * VEC, acc, VEC);
 }
 
 // ------------------------------------------------------------- decode kernel
@@ -1226,6 +1412,56 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 }
             }
         }
+
+        if (a.fold_cnt != nullptr && cs.dest >= 0) {
+            // A piece of a split (sequence, head group): count it, and the
+            // warp that completes the count merges the group's rows -- the
+            // merge kernel's work, done where the last piece lands.  Every
+            // piece is visible before it is counted (fence, then atomic).
+            __threadfence();
+            __syncwarp();
+            int is_last = 0;
+            if (lane == 0) {
+                const int ntu = prefix[cs.seq + 1] - prefix[cs.seq];
+                const long long T = (long long)prefix[a.B] * a.npairs;
+                const long long W = a.total_warps;
+                const long long a0 = (long long)prefix[cs.seq] * a.npairs + (long long)cs.pair * ntu;
+                const long long first = ((a0 + 1) * W + T - 1) / T - 1;
+                const long long last = ((a0 + ntu) * W + T - 1) / T - 1;
+                // warps whose range meets the pair's tiles; with fewer tiles
+                // than warps each range holds at most one tile
+                const long long expected = T >= W ? last - first + 1 : ntu;
+                is_last = atomicAdd(a.fold_cnt + (size_t)cs.seq * a.npairs + cs.pair, 1) == expected - 1;
+            }
+            is_last = __shfl_sync(FULL, is_last, 0);
+            if (is_last) {
+                __threadfence();
+                MergeArgs ma;
+                ma.out = a.out;
+                ma.context_lens = a.context_lens;
+                ma.prefix = prefix;
+                ma.part_o = a.part_o;
+                ma.part_m = a.part_m;
+                ma.part_l = a.part_l;
+                ma.mb = a.mb;
+                ma.B = a.B;
+                ma.Hq = a.Hq;
+                ma.G = a.G;
+                ma.n_hg = a.n_hg;
+                ma.npairs = a.npairs;
+                ma.bs = a.bs;
+                ma.hpu = HPU;
+                ma.mode = a.mode;
+                ma.part_tiles = a.part_tiles;
+                ma.S = a.S;
+                ma.total_warps = a.total_warps;
+                for (int g = 0; g < rows; ++g) {
+                    const MergeRow mr = merge_row(ma, (long long)cs.seq * a.Hq + h0 + g);
+                    if (mr.count > 1)  // small batches: few registers beside the decode loop's
+                        merge_row_warp<D, BF16, 4>(ma, mr);
+                }
+            }
+        }
     }
 
     if (failed) {
@@ -1239,186 +1475,18 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
     }
 }
 
+// Zero the decode kernel's per-row piece counters of this call.  Launched as
+// a programmatic dependent: it waits for the previous kernel in the stream
+// (which may still count with them) and lets the decode kernel's prologue
+// start at once.
+__global__ void __launch_bounds__(256) fold_zero_kernel(int *__restrict__ cnt, int n) {
+    griddep_launch_dependents();
+    griddep_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        cnt[i] = 0;
+}
+
 // ------------------------------------------------------------- merge kernel
-
-struct MergeArgs {
-    uint16_t *out;
-    const int32_t *context_lens;
-    const int32_t *prefix;   // balanced: tile prefix written by the decode kernel
-    const float *part_o, *part_m, *part_l;
-    int64_t mb;
-    int B, Hq, G, n_hg, npairs, bs;
-    int hpu;                 // query heads per decode unit (8 or 16)
-    int mode, part_tiles, S, total_warps;
-};
-// Balanced mode: prefix[B + 1] holds an upper bound on the pieces per row;
-// partition mode: S is the bound.
-
-constexpr int kMergeThreads = 128;
-constexpr int kMergeWideThreads = 512;  // one row per CTA, many pieces per row
-
-template <int NTH>
-__device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
-    constexpr unsigned FULL = 0xffffffffu;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float x = __shfl_xor_sync(FULL, v, o);
-        v = is_max ? fmaxf(v, x) : v + x;
-    }
-    const int warp = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) == 0)
-        red[warp] = v;
-    __syncthreads();
-    float r = red[0];
-#pragma unroll
-    for (int w = 1; w < NTH / 32; ++w)
-        r = is_max ? fmaxf(r, red[w]) : r + red[w];
-    __syncthreads();
-    return r;
-}
-
-// Where the pieces of one query head's split context are.
-struct MergeRow {
-    int seq, h, g;
-    long long count;   // pieces; <= 1 means nothing to merge
-    long long first;   // balanced: first warp
-    long long a0, T;   // balanced: flattened start of the pair, total tiles
-};
-
-__device__ __forceinline__ MergeRow merge_row(const MergeArgs &a, long long row) {
-    MergeRow r;
-    r.seq = (int)(row / a.Hq);
-    r.h = (int)(row - (long long)r.seq * a.Hq);
-    const int kvh = r.h / a.G;
-    const int hl = r.h - kvh * a.G;
-    const int hg = hl / a.hpu;
-    r.g = hl - hg * a.hpu;
-    const int pair = kvh * a.n_hg + hg;
-    r.first = 0;
-    r.a0 = 0;
-    r.T = 1;
-    if (a.mode == kModePartition) {
-        int c = a.context_lens[r.seq];
-        const int64_t cap = a.mb * a.bs;
-        c = c < 0 ? 0 : (c > cap ? (int)cap : c);
-        const int nt = (c + kTileTokens - 1) / kTileTokens;
-        r.count = (nt + a.part_tiles - 1) / a.part_tiles;  // <= 1: written by the decode kernel
-    } else {
-        const int nt = a.prefix[r.seq + 1] - a.prefix[r.seq];
-        r.count = 0;
-        if (nt > 0) {
-            r.T = (long long)a.prefix[a.B] * a.npairs;
-            r.a0 = (long long)a.prefix[r.seq] * a.npairs + (long long)pair * nt;
-            const long long W = a.total_warps;
-            r.first = ((r.a0 + 1) * W + r.T - 1) / r.T - 1;                 // warp holding a0
-            const long long last = ((r.a0 + nt) * W + r.T - 1) / r.T - 1;  // warp holding a0+nt-1
-            r.count = last - r.first + 1;  // 1: the pair sat in one warp, already final
-        }
-    }
-    return r;
-}
-
-// Partial row of piece k, or -1 (a warp whose range is empty).
-__device__ __forceinline__ long long merge_piece(const MergeArgs &a, const MergeRow &r, long long k) {
-    if (a.mode == kModePartition)
-        return ((long long)r.seq * a.Hq + r.h) * a.S + k;
-    const long long w = r.first + k;
-    if (r.T >= a.total_warps) {
-        // no warp has an empty range: the first piece is the first warp's
-        // last segment (slot 1), every later piece its warp's first (slot 0)
-        return (2 * w + (k == 0 ? 1 : 0)) * kMaxRows + r.g;
-    }
-    const long long lo = w * r.T / a.total_warps;
-    const long long hi = (w + 1) * r.T / a.total_warps;
-    if (lo >= hi)
-        return -1;
-    return (2 * w + (r.a0 < lo ? 0 : 1)) * kMaxRows + r.g;
-}
-
-template <int D, bool BF16>
-__device__ __forceinline__ void store_row(const MergeArgs &a, const MergeRow &r, int c, const float *v,
-                                          int n) {
-    uint32_t *dst = reinterpret_cast<uint32_t *>(a.out + ((size_t)r.seq * a.Hq + r.h) * D + c);
-    for (int i = 0; i < n / 2; ++i)
-        dst[i] = pack2<BF16>(v[2 * i], v[2 * i + 1]);
-}
-
-constexpr int kWarpPieces = 64;  // rows with at most this many pieces: one warp each
-
-// One warp merges one row, kWarpBatch pieces at a time (rescaled online
-// across batches).  A piece's output row does not depend on its weight, so
-// each batch issues every load at once: lane j < kWarpBatch fetches piece
-// j's (m, l), every lane its D/32 columns of all the batch's outputs; the
-// reductions are shuffles.  One memory round trip per batch.
-constexpr int kWarpBatch = 16;
-
-template <int D, bool BF16>
-__device__ __forceinline__ void merge_row_warp(const MergeArgs &a, const MergeRow &r) {
-    constexpr unsigned FULL = 0xffffffffu;
-    constexpr int VEC = D / 32;
-    const int lane = threadIdx.x & 31;
-    float M = -INFINITY, L = 0.f;
-    float acc[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i)
-        acc[i] = 0.f;
-    for (long long k0 = 0; k0 < r.count; k0 += kWarpBatch) {
-        const long long kl = k0 + lane;
-        const long long rl = (lane < kWarpBatch && kl < r.count) ? merge_piece(a, r, kl) : -1;
-        const float ml = rl >= 0 ? a.part_m[rl] : -INFINITY;
-        const float ll = rl >= 0 ? a.part_l[rl] : 0.f;
-        float v[kWarpBatch][VEC];
-#pragma unroll
-        for (int j = 0; j < kWarpBatch; ++j) {
-            const long long rr = __shfl_sync(FULL, rl, j);
-#pragma unroll
-            for (int i = 0; i < VEC; ++i)
-                v[j][i] = 0.f;
-            if (rr >= 0) {  // an empty piece (-1) has no row
-                const float *p = a.part_o + rr * D + lane * VEC;
-                if constexpr (VEC == 4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(p);
-                    v[j][0] = x.x;
-                    v[j][1 % VEC] = x.y;
-                    v[j][2 % VEC] = x.z;
-                    v[j][3 % VEC] = x.w;
-                } else {
-                    const float2 x = *reinterpret_cast<const float2 *>(p);
-                    v[j][0] = x.x;
-                    v[j][1 % VEC] = x.y;
-                }
-            }
-        }
-        float cm = ml;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
-        const float mnew = fmaxf(M, cm);
-        const float rescale = M == -INFINITY ? 0.f : exp2f(M - mnew);
-        const float w = ml == -INFINITY ? 0.f : exp2f(ml - mnew);
-        float lsum = w * ll;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            lsum += __shfl_xor_sync(FULL, lsum, o);
-        L = L * rescale + lsum;
-        M = mnew;
-#pragma unroll
-        for (int i = 0; i < VEC; ++i)
-            acc[i] *= rescale;
-#pragma unroll
-        for (int j = 0; j < kWarpBatch; ++j) {
-            const float wj = __shfl_sync(FULL, w, j);
-#pragma unroll
-            for (int i = 0; i < VEC; ++i)
-                acc[i] = wj != 0.f ? fmaf(wj, v[j][i], acc[i]) : acc[i];
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-    for (int i = 0; i < VEC; ++i)
-        acc[i] *= inv;
-    store_row<D, BF16>(a, r, lane * VEC, acc, VEC);
-}
 
 // The whole CTA merges one row with many pieces, GROUPS * kCtaBatch pieces
 // per batch (rescaled online across batches): thread (grp, col) owns one

@@ -412,9 +412,9 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
 // Workspace layout.
 //  partition: part_o [B][Hq][S][D] f32 | part_m [B][Hq][S] f32 | part_l [B][Hq][S] f32
 //  balanced:  prefix [B+1] i32 + pieces bound (256-aligned) | part_m [2W][16] | part_l [2W][16] | part_o [2W][16][D]
-//             with W = the largest warp count a launch may use.
+//             | piece counters [B][npairs] i32, with W = the largest warp count a launch may use.
 struct WsLayout {
-    size_t prefix = 0, m = 0, l = 0, o = 0, total = 0;
+    size_t prefix = 0, m = 0, l = 0, o = 0, cnt = 0, total = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -433,7 +433,8 @@ WsLayout ws_layout(const Plan &p, int64_t B, int64_t Hq, int64_t D, int64_t max_
         w.m = align256((size_t)(B + 2) * 4);
         w.l = align256(w.m + slots * kMaxRows * 4);
         w.o = align256(w.l + slots * kMaxRows * 4);
-        w.total = align256(w.o + slots * kMaxRows * D * 4);
+        w.cnt = align256(w.o + slots * kMaxRows * D * 4);  // piece counters [B][npairs]
+        w.total = align256(w.cnt + (size_t)B * p.npairs * 4);
     }
     return w;
 }
@@ -696,6 +697,15 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.part_m = have_ws ? reinterpret_cast<float *>(ws + wl.m) : nullptr;
     a.part_l = have_ws ? reinterpret_cast<float *>(ws + wl.l) : nullptr;
     a.prefix_out = have_ws ? reinterpret_cast<int32_t *>(ws + wl.prefix) : nullptr;
+    // Balanced schedules with one or two query heads per KV head merge split
+    // rows in the decode kernel itself (the last piece of a row merges it,
+    // saving the merge kernel's launch); with more heads per unit the last
+    // warp's serial merge of every head lands on the kernel's tail and the
+    // merge kernel is faster (measured: 13B-shaped 215.0 -> 211.7 us,
+    // 70B-shaped 89.8 -> 108.0 us).  PKV_FOLD_MERGE=0 / 1 forces it off / on.
+    const int fold_env = env_int("PKV_FOLD_MERGE", -1);
+    const bool fold = p.mode == kModeBalanced && (fold_env < 0 ? p.G <= 2 : fold_env != 0);
+    a.fold_cnt = fold ? reinterpret_cast<int *>(ws + wl.cnt) : nullptr;
     a.total_warps = p.total_warps;
     a.stages = p.stages;
     a.err = err;
@@ -720,6 +730,12 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     DecodeKernel k = pick_decode((int)D, bf16, p.nt, fp8, p.fma, cas != nullptr);
     if (!k)
         return PKV_ERR_INVALID;
+    if (fold) {
+        const int n = (int)(num_seqs * p.npairs);
+        if (!cuda_ok(launch_dependent(fold_zero_kernel, dim3((unsigned)std::min(148, (n + 255) / 256)), dim3(256), 0,
+                                      (cudaStream_t)stream, a.fold_cnt, n)))
+            return PKV_ERR_CUDA;
+    }
     if (cas) {
         // the cascade instantiation shares the plan of the plain kernel; give
         // it the same shared-memory ceiling once per device
@@ -739,7 +755,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
                                   tmV, a)))
         return PKV_ERR_CUDA;
 
-    const bool merge = (p.mode == kModeBalanced) || (p.mode == kModePartition && p.S > 1);
+    const bool merge = (p.mode == kModeBalanced && !fold) || (p.mode == kModePartition && p.S > 1);
     if (merge) {
         MergeArgs m;
         m.out = a.out;
