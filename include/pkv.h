@@ -429,12 +429,14 @@ pkv_status pkv_batch_tables(void *h, const int32_t *seqs, int32_t n, int32_t *ds
                             int32_t cap, int32_t *context_lens);
 
 /* Sharing groups of a batch (host), for
- * pkv_append_decode_attention_shared_prefix: consecutive sequences of
- * seqs[0..n) whose first block is one and the same shared block (refcount >
- * 1) form a group, any other sequence a group of its own.  group_start[0 ..
- * *num_groups] receives the groups (capacity n + 1), shared_lens[i] the
- * number of leading positions of seqs[i] held in shared blocks (its leading
- * blocks with refcount > 1, times bs). */
+ * pkv_append_decode_attention_shared_prefix: runs of consecutive sequences
+ * of seqs[0..n) whose first block, where it is shared (refcount > 1), is one
+ * and the same block; a sequence that shares nothing stays in the run around
+ * it (a member with claim 0) rather than splitting it, since each group reads
+ * its prefix once.  A sequence whose shared first block differs from the
+ * run's opens a new group.  group_start[0 .. *num_groups] receives the groups
+ * (capacity n + 1), shared_lens[i] the number of leading positions of seqs[i]
+ * held in shared blocks (its leading blocks with refcount > 1, times bs). */
 pkv_status pkv_batch_prefix_groups(void *h, const int32_t *seqs, int32_t n, int32_t *group_start,
                                    int32_t *num_groups, int32_t *shared_lens);
 

@@ -354,16 +354,23 @@ pkv_status pkv_batch_prefix_groups(void *h, const int32_t *seqs, int32_t n, int3
     for (int32_t i = 0; i < n; ++i)
         if (!a->valid_seq(seqs[i]))
             return PKV_ERR_INVALID;
+    // A sequence that shares nothing joins the open group as a member with
+    // claim 0 instead of splitting it: split groups would each read the
+    // common prefix again.  A sequence whose first block is shared joins when
+    // the open group has that first block, or none yet; otherwise it opens a
+    // new group.
     int32_t ng = 0;
-    int32_t group_first = -1;  // first block shared by the open group, -1: none
+    int32_t group_first = -1;  // first block shared by the open group, -1: none yet
     for (int32_t i = 0; i < n; ++i) {
         const Sequence &q = a->seqs[seqs[i]];
         const int32_t first = q.blocks.empty() ? -1 : q.blocks[0];
         const bool shared_first = first >= 0 && a->refcount[first] > 1;
-        if (i == 0 || !shared_first || first != group_first) {
+        if (i == 0 || (shared_first && group_first >= 0 && first != group_first)) {
             group_start[ng++] = i;
-            group_first = shared_first ? first : -1;
+            group_first = -1;
         }
+        if (shared_first)
+            group_first = first;
         size_t k = 0;
         while (k < q.blocks.size() && a->refcount[q.blocks[k]] > 1)
             ++k;

@@ -75,6 +75,11 @@ struct DecodeArgs {
     // warp that finishes the last piece of a split row merges it (no merge
     // kernel).  Null: the merge kernel does it.
     int *fold_cnt;
+    // balanced: every (sequence, head group) with work weighs its tiles plus
+    // unit_cost virtual tiles at the end of its range (nothing is computed
+    // there), so that a warp given many short units gets fewer tiles: a unit
+    // costs a query load, a resume and an epilogue beside its tiles
+    int unit_cost;
     int total_warps;
     int stages;
     unsigned *err;
@@ -199,13 +204,25 @@ __device__ __forceinline__ void walker_init(Walker &w, const DecodeArgs &a, cons
         w.hi = range_lo(gw + 1, T, a.total_warps);
         w.u = w.lo;
         if (w.lo < w.hi) {
+            // the range may start in a pair's virtual tail: the walker skips it
             int s = upper_bound_i(prefix, a.B + 1, w.lo / a.npairs) - 1;
-            const int nt = prefix[s + 1] - prefix[s];
+            const int ws = prefix[s + 1] - prefix[s];
             const long long r = w.lo - (long long)prefix[s] * a.npairs;
             w.seq = s;
-            w.pair = (int)(r / nt);
-            w.t = (int)(r % nt);
+            w.pair = (int)(r / ws);
+            w.t = (int)(r % ws);
         }
+    }
+}
+
+// balanced: from the end of a pair's span to the start of the next pair with work
+__device__ __forceinline__ void walker_next_pair(Walker &w, const DecodeArgs &a, const int *prefix) {
+    w.t = 0;
+    if (++w.pair == a.npairs) {
+        w.pair = 0;
+        ++w.seq;
+        while (w.seq < a.B && prefix[w.seq + 1] == prefix[w.seq])
+            ++w.seq;
     }
 }
 
@@ -253,30 +270,35 @@ __device__ __forceinline__ bool walker_next_raw(Walker &w, Seg &sg, const Decode
         w.u += a.total_warps;
         return true;
     }
-    // balanced
-    if (w.u >= w.hi)
-        return false;
-    const int nt = prefix[w.seq + 1] - prefix[w.seq];
-    sg.seq = w.seq;
-    sg.pair = w.pair;
-    sg.ctx = ctxs[w.seq];
-    sg.t0 = w.t;
-    sg.t1 = (int)min((long long)nt, (long long)w.t + (w.hi - w.u));
-    const long long pair_start = (long long)prefix[w.seq] * a.npairs + (long long)w.pair * nt;
-    const bool complete = (sg.t0 == 0 && sg.t1 == nt);
-    sg.dest = complete ? -1 : 2 * gw + (pair_start < w.lo ? 0 : 1);
-    w.u += sg.t1 - sg.t0;
-    w.t = sg.t1;
-    if (w.t == nt) {
-        w.t = 0;
-        if (++w.pair == a.npairs) {
-            w.pair = 0;
-            ++w.seq;
-            while (w.seq < a.B && prefix[w.seq + 1] == prefix[w.seq])
-                ++w.seq;
+    // balanced: pair p of sequence s spans ws = nt + unit_cost positions of
+    // the flattened order, its nt real tiles first
+    for (;;) {
+        if (w.u >= w.hi)
+            return false;
+        const int ws = prefix[w.seq + 1] - prefix[w.seq];
+        const int nt = ws - a.unit_cost;
+        if (w.t >= nt) {
+            // a range that starts in a pair's virtual tail: step over it
+            w.u += ws - w.t;
+            walker_next_pair(w, a, prefix);
+            continue;
         }
+        sg.seq = w.seq;
+        sg.pair = w.pair;
+        sg.ctx = ctxs[w.seq];
+        sg.t0 = w.t;
+        sg.t1 = (int)min((long long)nt, (long long)w.t + (w.hi - w.u));
+        const long long pair_start = (long long)prefix[w.seq] * a.npairs + (long long)w.pair * ws;
+        const bool complete = (sg.t0 == 0 && sg.t1 == nt);
+        sg.dest = complete ? -1 : 2 * gw + (pair_start < w.lo ? 0 : 1);
+        w.u += sg.t1 - sg.t0;
+        w.t = sg.t1;
+        if (w.t == nt) {
+            w.u += ws - nt;
+            walker_next_pair(w, a, prefix);
+        }
+        return true;
     }
-    return true;
 }
 
 // ------------------------------------------------------------- conversions
@@ -325,7 +347,18 @@ struct MergeArgs {
     int B, Hq, G, n_hg, npairs, bs;
     int hpu;                 // query heads per decode unit (8 or 16)
     int mode, part_tiles, S, total_warps;
+    int unit_cost;           // balanced: virtual tiles per pair (decode kernel's)
 };
+
+// Balanced: where pair `pair` of sequence `seq` sits in the flattened order:
+// its first position a0 and its real tiles nt (0: no work), the pair's span
+// being nt + unit_cost positions.
+__device__ __forceinline__ void pair_span(const int32_t *prefix, int seq, int pair, int npairs, int unit_cost,
+                                          long long &a0, int &nt) {
+    const int ws = prefix[seq + 1] - prefix[seq];
+    nt = ws > 0 ? ws - unit_cost : 0;
+    a0 = (long long)prefix[seq] * npairs + (long long)pair * ws;
+}
 // Balanced mode: prefix[B + 1] holds an upper bound on the pieces per row;
 // partition mode: S is the bound.
 
@@ -379,11 +412,11 @@ __device__ __forceinline__ MergeRow merge_row(const MergeArgs &a, long long row)
         const int nt = (c + kTileTokens - 1) / kTileTokens;
         r.count = (nt + a.part_tiles - 1) / a.part_tiles;  // <= 1: written by the decode kernel
     } else {
-        const int nt = a.prefix[r.seq + 1] - a.prefix[r.seq];
+        int nt;
+        pair_span(a.prefix, r.seq, pair, a.npairs, a.unit_cost, r.a0, nt);
         r.count = 0;
         if (nt > 0) {
             r.T = (long long)a.prefix[a.B] * a.npairs;
-            r.a0 = (long long)a.prefix[r.seq] * a.npairs + (long long)pair * nt;
             const long long W = a.total_warps;
             r.first = ((r.a0 + 1) * W + r.T - 1) / r.T - 1;                 // warp holding a0
             const long long last = ((r.a0 + nt) * W + r.T - 1) / r.T - 1;  // warp holding a0+nt-1
@@ -569,7 +602,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             const int c = clamp_ctx(__ldg(a.context_lens + s), a);
             ctxs[s] = c;
             const int nt = ceil_div_i(c, kTileTokens);
-            local += a.mode == kModeBalanced ? nt : ceil_div_i(nt, a.part_tiles);
+            local += a.mode == kModeBalanced ? (nt > 0 ? nt + a.unit_cost : 0) : ceil_div_i(nt, a.part_tiles);
         }
         // block-wide exclusive scan of `local`
         int incl = local;
@@ -590,7 +623,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
         for (int s = beg; s < end; ++s) {
             prefix[s] = run;
             const int nt = ceil_div_i(ctxs[s], kTileTokens);
-            run += a.mode == kModeBalanced ? nt : ceil_div_i(nt, a.part_tiles);
+            run += a.mode == kModeBalanced ? (nt > 0 ? nt + a.unit_cost : 0) : ceil_div_i(nt, a.part_tiles);
         }
         if (threadIdx.x == 0) {
             int tot = 0;
@@ -1422,10 +1455,11 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
             __syncwarp();
             int is_last = 0;
             if (lane == 0) {
-                const int ntu = prefix[cs.seq + 1] - prefix[cs.seq];
+                long long a0;
+                int ntu;
+                pair_span(prefix, cs.seq, cs.pair, a.npairs, a.unit_cost, a0, ntu);
                 const long long T = (long long)prefix[a.B] * a.npairs;
                 const long long W = a.total_warps;
-                const long long a0 = (long long)prefix[cs.seq] * a.npairs + (long long)cs.pair * ntu;
                 const long long first = ((a0 + 1) * W + T - 1) / T - 1;
                 const long long last = ((a0 + ntu) * W + T - 1) / T - 1;
                 // warps whose range meets the pair's tiles; with fewer tiles
@@ -1455,6 +1489,7 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 ma.part_tiles = a.part_tiles;
                 ma.S = a.S;
                 ma.total_warps = a.total_warps;
+                ma.unit_cost = a.unit_cost;
                 for (int g = 0; g < rows; ++g) {
                     const MergeRow mr = merge_row(ma, (long long)cs.seq * a.Hq + h0 + g);
                     if (mr.count > 1)  // small batches: few registers beside the decode loop's

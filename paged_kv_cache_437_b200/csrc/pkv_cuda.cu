@@ -267,6 +267,17 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
 
 // Plans depend only on the shape, the device and two tuning variables; they
 // are cached so that a steady decode loop pays no occupancy queries.
+// Balanced schedules: virtual tiles weighed per (sequence, head group), the
+// unit's fixed cost (query load, resume, epilogue) in tile-equivalents.  A
+// batch of many one- and two-tile units (the suffixes left after a shared
+// prefix) otherwise gives the warps that draw them several times the work of
+// the warps that stream long units.  PKV_UNIT_COST overrides it (0..8).
+constexpr int kMaxUnitCost = 8;
+int unit_cost() {
+    const int v = env_int("PKV_UNIT_COST", 3);
+    return v < 0 ? 0 : (v > kMaxUnitCost ? kMaxUnitCost : v);
+}
+
 struct PlanKey {
     int dev, warps_env, stages_env, fma_env;
     int64_t B, Hq, Hkv, D, max_ctx;
@@ -351,7 +362,7 @@ pkv_status make_plan_uncached(Plan &p, int64_t B, int64_t Hq, int64_t Hkv, int64
     }
     const bool need_prefix = p.mode != kModeDirect;
     // the on-chip schedule keeps per-sequence tile counts in int32
-    if (need_prefix && B * ceil_div64(max_ctx, kTileTokens) * p.npairs >= (int64_t(1) << 31))
+    if (need_prefix && B * (ceil_div64(max_ctx, kTileTokens) + kMaxUnitCost) * p.npairs >= (int64_t(1) << 31))
         return PKV_ERR_INVALID;
     for (;;) {
         SmemLayout L = decode_smem_layout((int)B, p.warps, p.stages, (int)D, need_prefix, fp8, p.fma);
@@ -706,6 +717,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     const int fold_env = env_int("PKV_FOLD_MERGE", -1);
     const bool fold = p.mode == kModeBalanced && (fold_env < 0 ? p.G <= 2 : fold_env != 0);
     a.fold_cnt = fold ? reinterpret_cast<int *>(ws + wl.cnt) : nullptr;
+    a.unit_cost = p.mode == kModeBalanced ? unit_cost() : 0;
     a.total_warps = p.total_warps;
     a.stages = p.stages;
     a.err = err;
@@ -776,6 +788,7 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
         m.part_tiles = p.part_tiles;
         m.S = p.S;
         m.total_warps = p.total_warps;
+        m.unit_cost = a.unit_cost;
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -271,15 +271,24 @@ def test_batch_prefix_groups():
         a.append_slot(p2)
     m3 = a.seq_fork(p2, 1)
     a.append_slot(m3)
-    # groups: runs of consecutive sequences whose first block is one shared block
+    # groups: runs of consecutive sequences whose shared first block is one
+    # and the same; `lone` shares nothing and stays in the run around it
     starts, shared = a.prefix_groups([p1, m1, m2, lone, m3, p2])
-    assert starts.tolist() == [0, 3, 4, 6]
+    assert starts.tolist() == [0, 4, 6]
     # claims: leading blocks with refcount > 1, times bs (p1's third block is
     # shared with m1 only; its fourth is private)
     assert shared.tolist() == [3 * bs, 3 * bs, 2 * bs, 0, bs, bs]
-    # a shared sequence separated from its group starts a new one
+    # a sequence sharing nothing does not split a group
     starts, _ = a.prefix_groups([m1, lone, m2])
+    assert starts.tolist() == [0, 3]
+    # ... and joins the group after it when it comes first
+    starts, _ = a.prefix_groups([lone, m3, p2])
+    assert starts.tolist() == [0, 3]
+    # a different shared first block opens a new group
+    starts, _ = a.prefix_groups([m1, m3, m2])
     assert starts.tolist() == [0, 1, 2, 3]
+    starts, _ = a.prefix_groups([lone])
+    assert starts.tolist() == [0, 1]
     starts, shared = a.prefix_groups([])
     assert starts.tolist() == [0] and shared.size == 0
     with pytest.raises(pkv.PkvError):

@@ -92,3 +92,16 @@ def test_named_workload_full_size(name):
         err = gh.assert_close(got, ref, w.spec.dtype, f"{name} mode {mode}")
         print(f"{name} mode {mode} fused {fused}: {len(ref) if pairs is not None else ref.size} compared, "
               f"max |err| {err:.3e}")
+
+
+@pytest.mark.parametrize("fold", ["0", "1"], ids=["merge_kernel", "merge_in_decode"])
+def test_split_rows_merged_either_way(small_case, fold, monkeypatch):
+    # the work-balanced schedule's split rows, merged by the merge kernel or
+    # by the decode kernel's last piece of each row (whichever the shape picks
+    # by default, both must agree with the oracle), plain and fused step
+    monkeypatch.setenv("PKV_FOLD_MERGE", fold)
+    w, kc, vc, slots, ref, k_ref, v_ref = small_case
+    for fused in (False, True):
+        step = gh.GpuStep(w, kc, vc, slots)
+        out = step.run_fused(pkv.PKV_PARTITION_AUTO) if fused else step.run(pkv.PKV_PARTITION_AUTO)
+        gh.assert_close(gh.to_f64(out), ref, w.spec.dtype, f"{w.spec.name} fold={fold} fused={fused}")

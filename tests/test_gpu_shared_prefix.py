@@ -104,9 +104,10 @@ def test_groups_from_the_allocator():
     starts, claims = alloc.prefix_groups(seqs)
     tables, lens = alloc.batch_tables(seqs, w.max_blocks_per_seq)
     alloc.close()
-    # the allocator's groups are the workload's (a sequence whose first block
-    # is private is a group of its own)
+    # the allocator's claims are the workload's; its groups are runs of one
+    # shared first block, with sequences that share nothing kept inside them
     assert np.array_equal(lens, w.context_lens)
+    assert starts[0] == 0 and starts[-1] == sp.num_seqs and np.all(np.diff(starts) > 0)
     for s in range(sp.num_seqs):
         assert claims[s] == w.shared_blocks[s] * sp.block_size
     # same attention on the allocator's own block ids: permute the pool into them
