@@ -80,23 +80,23 @@ struct MqArgs {
     int inject_no_issue;           // testing: issue no copies so that waits run out
 };
 
-// Shared-memory plan (from a 1024-aligned base): Q tile, K ring, V ring, P
-// tile, then barriers, small state and the per-sequence unit prefix.
+// Shared-memory plan (from a 1024-aligned base): Q tile, K ring, V ring,
+// then the exchange buffer, barriers, small state and the per-sequence unit
+// prefix.  P never touches shared memory: it is written to tensor memory over
+// its own scores and read from there by the P V product.
 template <int D>
 struct MqSmem {
     static constexpr int kTileBytes = kMqTile * D * 2;   // K or V tile; Q (128 rows) too
     static constexpr int kHalf = kMqTile * 128;          // one 128-byte column half of a tile
-    static constexpr int kPBytes = kMqRows * kMqTile * 2;
     static constexpr int q = 0;
     static constexpr int k = q + kTileBytes;
     static constexpr int v = k + kMqKStages * kTileBytes;
-    static constexpr int p = v + kMqVStages * kTileBytes;
-    static constexpr int xbuf = p + kPBytes;                // [2 parity][2 halves][128 rows] f32
+    static constexpr int xbuf = v + kMqVStages * kTileBytes;  // [2 parity][2 halves][128 rows] f32
     static constexpr int bars = xbuf + 2 * 2 * kMqRows * 4;
     // barrier indices
     static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kMqKStages,
                          kVFull = kKEmpty + kMqKStages, kVEmpty = kVFull + kMqVStages, kSFull = kVEmpty + kMqVStages,
-                         kSFree = kSFull + 2, kPFull = kSFree + 2, kODone = kPFull + 1, kUnitFull = kODone + 1,
+                         kSFree = kSFull + 2, kPFull = kSFree + 2, kODone = kPFull + 2, kUnitFull = kODone + 1,
                          kUnitEmpty = kUnitFull + 2, kDrain = kUnitEmpty + 2, kXch = kDrain + 1,
                          kNumBars = kXch + 4;
     static constexpr int misc = bars + kNumBars * 8;     // [0..1] unit slots, [2] TMEM base, [3] abort
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base + L::q, sK = base + L::k, sV = base + L::v, sP = base + L::p;
+    const uint32_t sQ = base + L::q, sK = base + L::k, sV = base + L::v;
     auto bar = [&](int i) { return base + (uint32_t)(L::bars + i * 8); };
     volatile int *misc = reinterpret_cast<volatile int *>(gbase + L::misc);
     int *prefix = reinterpret_cast<int *>(gbase + L::prefix);
@@ -247,11 +247,12 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(L::kSFull + i), 1);
-            mbar_init(bar(L::kSFree + i), kMqSoftmaxWarps);      // one arrival per softmax warp
+            mbar_init(bar(L::kSFree + i), 1);  // P V of the buffer's last tile is done (its P is read)
             mbar_init(bar(L::kUnitFull + i), 1);
             mbar_init(bar(L::kUnitEmpty + i), 2 + kMqSoftmaxWarps);  // MMA thread, V producer, softmax warps
         }
-        mbar_init(bar(L::kPFull), kMqSoftmaxWarps);
+        for (int i = 0; i < 2; ++i)
+            mbar_init(bar(L::kPFull + i), kMqSoftmaxWarps);  // P of tiles of this parity: one arrival per softmax warp
         for (int i = 0; i < 4; ++i)
             mbar_init(bar(L::kXch + i), 2);  // the two warps of a 32-row quarter
         mbar_init(bar(L::kODone), 1);
@@ -454,24 +455,30 @@ __global__ void __launch_bounds__(kMqThreads, 1)
             bool ok = true, issued = false;
             auto issue_pv = [&](uint32_t jp, bool first) {
                 const int vt = (int)(jp % VS);
-                if (!mq_wait(bar(L::kPFull), jp & 1, a, abort_flag) ||
+                if (!mq_wait(bar(L::kPFull + (jp & 1)), (jp >> 1) & 1, a, abort_flag) ||
                     !mq_wait(bar(L::kVFull + vt), (jp / VS) & 1, a, abort_flag))
                     return false;
                 tc_fence_after();
                 // O_h += P_h V_h for the two 64-position halves h of the tile:
                 // each softmax half keeps its own running max, so each has its
-                // own accumulator (combined once per unit in the epilogue)
+                // own accumulator (combined once per unit in the epilogue).
+                // P_h sits in tensor memory over the first 32 columns of the
+                // half's scores (16-bit pairs, one row per lane); a k-step of
+                // 16 positions is 8 columns.
+                const uint32_t p_cols = tmem + (jp & 1) * kMqTile;
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int ks = 0; ks < kMqTile / 32; ++ks) {
-                        const uint64_t ad = smem_desc_sw128(sP + h * kHalf + ks * 32, 16, 1024);
                         const uint64_t bd =
                             smem_desc_sw128(sV + vt * kTileBytes + h * (kMqTile / 2) * 128 + ks * 2048, kHalf, 1024);
-                        tc_mma_ss(tmem + kColO + h * D, ad, bd, idesc_o, (first && ks == 0) ? 0u : 1u);
+                        tc_mma_ts(tmem + kColO + h * D, p_cols + h * (kMqTile / 2) + ks * 8, bd, idesc_o,
+                                  (first && ks == 0) ? 0u : 1u);
                     }
                 tc_commit(bar(L::kODone));
                 tc_commit(bar(L::kVEmpty + vt));
+                // the score buffer (holding P) may take the scores of tile jp + 2
+                tc_commit(bar(L::kSFree + (jp & 1)));
                 return true;
             };
             while (ok) {
@@ -598,26 +605,17 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 if (!ok)
                     break;
                 tc_fence_after();
+                // (S_j complete means P V of tile j - 2 is done: the arrival
+                // below lands in the phase of tile j of this parity's P_full)
+                const bool ragged = (j + 1) * kMqTile > U.ctx;
                 if (!warp_active) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(bar(L::kSFree + (jg & 1)));
                     if (!(ok = zero_v_tail(j)))
                         break;
-                    // arrive for this tile only once the previous tile's
-                    // phase is complete (its P V has run): a padding warp must
-                    // not run ahead of the others into the next phase
-                    if (jg > 0) {
-                        ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
-                        if (!ok)
-                            break;
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
+                    if (ragged)
+                        fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(bar(L::kPFull));
+                        mbar_arrive(bar(L::kPFull + (jg & 1)));
                     continue;
                 }
                 uint32_t sv[HC];
@@ -626,10 +624,6 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                     tmem_ld32(lane_base + (jg & 1) * kMqTile + hc * HC + c * 32,
                               *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
                 tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(bar(L::kSFree + (jg & 1)));
                 const int pos0 = j * kMqTile + hc * HC;
                 if (pos0 + HC > lim) {
 #pragma unroll
@@ -674,13 +668,22 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 const float2 r01 = f32x2_unpack(f32x2_add(rs2[0], rs2[1]));
                 const float2 r23 = f32x2_unpack(f32x2_add(rs2[2], rs2[3]));
                 l += (r01.x + r01.y) + (r23.x + r23.y);
-                if (j > 0) {
-                    // P V of the previous tile is done: P may be overwritten and O rescaled
+                // O_done of the previous tile is waited at every tile (before
+                // the rescale when there is one, else just before P_full's
+                // arrival): S_j complete means P V of tile jg - 2 is done, and
+                // P V of tile jg needs this warp's arrival, so the barrier is
+                // within one phase of the one waited for, as its parity test
+                // needs; the epilogue's wait for the last tile relies on it
+                bool o_prev = jg == 0;
+                if (j > 0 && __any_sync(FULL, need)) {
+                    // the reference max moved: O_hc is rescaled once the
+                    // previous tile's P V is in it
                     ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
                     if (!ok)
                         break;
+                    o_prev = true;
                     tc_fence_after();
-                    if (__any_sync(FULL, need)) {
+                    {
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
                             uint32_t o[32];
@@ -694,23 +697,21 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                         tmem_wait_st();
                     }
                 }
-                // P_hc -> shared memory, K-major 128-byte swizzle: positions
-                // 64 hc .. 64 hc + 63 of row r at sP + hc*kHalf + r*128, 16-byte
-                // chunk c at (c ^ (r % 8)) * 16
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t addr = sP + hc * kHalf + r * 128 + ((c ^ (r & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c * 4]),
-                                 "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
-                                 : "memory");
-                }
+                // P_hc -> tensor memory over this warp's own (already read)
+                // scores: positions 64 hc .. 64 hc + 63 of row r as 32
+                // columns of 16-bit pairs from column 64 hc of the buffer
+                tmem_st32(lane_base + (jg & 1) * kMqTile + hc * HC, *reinterpret_cast<uint32_t(*)[32]>(pk));
+                tmem_wait_st();
                 if (!(ok = zero_v_tail(j)))
                     break;
-                fence_proxy_async_smem();
+                if (ragged)
+                    fence_proxy_async_smem();
+                if (!o_prev && !(ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag))))
+                    break;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(bar(L::kPFull));
+                    mbar_arrive(bar(L::kPFull + (jg & 1)));
             }
             if (!ok)
                 break;
@@ -722,6 +723,8 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 ++k;
                 continue;
             }
+            // O holds every tile once the last P V is done (the one before it
+            // was waited at the last tile)
             ok = __all_sync(FULL, mq_wait(bar(L::kODone), (jg - 1) & 1, a, abort_flag));
             if (!ok)
                 break;
