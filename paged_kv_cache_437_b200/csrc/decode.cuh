@@ -451,6 +451,84 @@ __device__ __forceinline__ void store_row(const MergeArgs &a, const MergeRow &r,
         dst[i] = pack2<BF16>(v[2 * i], v[2 * i + 1]);
 }
 
+// All `rows` query heads of one split (sequence, head group) merged by one
+// warp at once: the heads share their pieces (the same warps computed them),
+// and a piece's rows are contiguous (partial row base + g).  Lane l takes head
+// g = l / (32 / rp) (rp = rows rounded up to a power of two) and D / (32 / rp)
+// of its columns, 16 at a time.  First pass: each head's M over the pieces;
+// second: weights 2^(m_k - M) and the weighted sums.  Every load of a pass
+// is independent, so the merge costs two or three memory round trips instead
+// of one per piece batch per head.
+constexpr int kPairMergeMaxPieces = 16;
+
+template <int D, bool BF16>
+__device__ __forceinline__ void merge_pair_warp(const MergeArgs &a, const MergeRow &r0, int rows) {
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int CH = 16;  // columns per lane per pass
+    const int lane = threadIdx.x & 31;
+    int rp = 1;
+    while (rp < rows)
+        rp <<= 1;
+    const int lpr = 32 / rp;          // lanes per head
+    const int g = lane / lpr;
+    const int cpl = D / lpr;          // columns per lane (>= 4)
+    const int c_lane = (lane - g * lpr) * cpl;
+    const bool on = g < rows;
+    const int n = (int)r0.count;
+    // piece k's partial row base (of head 0 of the group), -1 for an empty piece
+    long long base[kPairMergeMaxPieces];
+#pragma unroll
+    for (int k = 0; k < kPairMergeMaxPieces; ++k)
+        base[k] = k < n ? merge_piece(a, r0, k) - r0.g : -1;
+    float mk[kPairMergeMaxPieces];
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kPairMergeMaxPieces; ++k) {
+        mk[k] = (on && base[k] >= 0) ? a.part_m[base[k] + g] : -INFINITY;
+        M = fmaxf(M, mk[k]);
+    }
+    float L = 0.f;
+#pragma unroll
+    for (int k = 0; k < kPairMergeMaxPieces; ++k) {
+        mk[k] = mk[k] == -INFINITY ? 0.f : exp2f(mk[k] - M);  // the piece's weight
+        if (mk[k] != 0.f)
+            L = fmaf(mk[k], a.part_l[base[k] + g], L);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    MergeRow rg = r0;
+    rg.h = r0.h + g;
+    for (int c0 = 0; c0 < cpl; c0 += CH) {
+        const int nc = cpl - c0 < CH ? cpl - c0 : CH;  // 4, 8 or 16
+        float acc[CH];
+#pragma unroll
+        for (int i = 0; i < CH; ++i)
+            acc[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kPairMergeMaxPieces; ++k) {
+            if (mk[k] == 0.f)
+                continue;
+            const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (base[k] + g) * D + c_lane + c0);
+#pragma unroll
+            for (int i = 0; i < CH / 4; ++i) {
+                if (4 * i < nc) {
+                    const float4 x = src[i];
+                    acc[4 * i] = fmaf(mk[k], x.x, acc[4 * i]);
+                    acc[4 * i + 1] = fmaf(mk[k], x.y, acc[4 * i + 1]);
+                    acc[4 * i + 2] = fmaf(mk[k], x.z, acc[4 * i + 2]);
+                    acc[4 * i + 3] = fmaf(mk[k], x.w, acc[4 * i + 3]);
+                }
+            }
+        }
+        if (on) {
+#pragma unroll
+            for (int i = 0; i < CH; ++i)
+                acc[i] *= inv;
+            store_row<D, BF16>(a, rg, c_lane + c0, acc, nc);
+        }
+    }
+    __syncwarp(FULL);
+}
+
 constexpr int kWarpPieces = 64;  // rows with at most this many pieces: one warp each
 
 // One warp merges one row, kWarpBatch pieces at a time (rescaled online
@@ -1490,10 +1568,15 @@ __global__ void __launch_bounds__(256) paged_decode_kernel(const __grid_constant
                 ma.S = a.S;
                 ma.total_warps = a.total_warps;
                 ma.unit_cost = a.unit_cost;
-                for (int g = 0; g < rows; ++g) {
-                    const MergeRow mr = merge_row(ma, (long long)cs.seq * a.Hq + h0 + g);
-                    if (mr.count > 1)  // small batches: few registers beside the decode loop's
-                        merge_row_warp<D, BF16, 4>(ma, mr);
+                const MergeRow m0 = merge_row(ma, (long long)cs.seq * a.Hq + h0);
+                if (rows > 1 && m0.count <= kPairMergeMaxPieces) {
+                    merge_pair_warp<D, BF16>(ma, m0, rows);  // every head at once
+                } else {
+                    for (int g = 0; g < rows; ++g) {
+                        const MergeRow mr = merge_row(ma, (long long)cs.seq * a.Hq + h0 + g);
+                        if (mr.count > 1)  // small batches: few registers beside the decode loop's
+                            merge_row_warp<D, BF16, 4>(ma, mr);
+                    }
                 }
             }
         }

@@ -708,14 +708,16 @@ pkv_status decode_impl(const void *q, int64_t num_seqs, int64_t num_q_heads, pkv
     a.part_m = have_ws ? reinterpret_cast<float *>(ws + wl.m) : nullptr;
     a.part_l = have_ws ? reinterpret_cast<float *>(ws + wl.l) : nullptr;
     a.prefix_out = have_ws ? reinterpret_cast<int32_t *>(ws + wl.prefix) : nullptr;
-    // Balanced schedules with one or two query heads per KV head merge split
-    // rows in the decode kernel itself (the last piece of a row merges it,
-    // saving the merge kernel's launch); with more heads per unit the last
-    // warp's serial merge of every head lands on the kernel's tail and the
-    // merge kernel is faster (measured: 13B-shaped 215.0 -> 211.7 us,
-    // 70B-shaped 89.8 -> 108.0 us).  PKV_FOLD_MERGE=0 / 1 forces it off / on.
+    // Balanced schedules merge split rows in the decode kernel itself (the
+    // warp finishing a (sequence, head group)'s last piece merges all its
+    // heads at once), saving the merge kernel's launch, when rows are split
+    // into few pieces: at most ~4 warps per (sequence, head group) on average.
+    // Long rows split over many warps (one or two long sequences) keep the
+    // merge kernel, which spreads them over the whole GPU.  PKV_FOLD_MERGE=0
+    // / 1 forces it off / on.
     const int fold_env = env_int("PKV_FOLD_MERGE", -1);
-    const bool fold = p.mode == kModeBalanced && (fold_env < 0 ? p.G <= 2 : fold_env != 0);
+    const bool fold = p.mode == kModeBalanced &&
+                      (fold_env < 0 ? (int64_t)p.total_warps <= 4 * num_seqs * p.npairs : fold_env != 0);
     a.fold_cnt = fold ? reinterpret_cast<int *>(ws + wl.cnt) : nullptr;
     a.unit_cost = p.mode == kModeBalanced ? unit_cost() : 0;
     a.total_warps = p.total_warps;
