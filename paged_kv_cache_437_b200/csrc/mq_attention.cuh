@@ -477,8 +477,6 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                     }
                 tc_commit(bar(L::kODone));
                 tc_commit(bar(L::kVEmpty + vt));
-                // the score buffer (holding P) may take the scores of tile jp + 2
-                tc_commit(bar(L::kSFree + (jp & 1)));
                 return true;
             };
             while (ok) {
@@ -496,8 +494,10 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                     break;
                 for (int j = 0; j < U.nt; ++j, ++jg) {
                     const int st = (int)(jg % KS);
-                    ok = mq_wait(bar(L::kKFull + st), (jg / KS) & 1, a, abort_flag) &&
-                         mq_wait(bar(L::kSFree + (jg & 1)), ((jg >> 1) & 1) ^ 1, a, abort_flag);
+                    // (the score buffer of tile jg held P of tile jg - 2: the
+                    // P V that read it was issued before this S, and tcgen05
+                    // MMAs issued by one thread execute in issue order)
+                    ok = mq_wait(bar(L::kKFull + st), (jg / KS) & 1, a, abort_flag);
                     if (!ok)
                         break;
                     tc_fence_after();
