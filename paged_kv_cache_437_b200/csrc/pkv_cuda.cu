@@ -474,10 +474,14 @@ pkv_status mq_launch(MqArgs a, const void *q, int64_t nz, const pkv_cache &kc, c
         return PKV_ERR_CUDA;
     void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const MqArgs) = nullptr;
     int smem = 0;
-    // PKV_MQ_POLY=1: 3 of every 8 probability pairs by the FMA-pipe exp2
-    const bool poly = env_int("PKV_MQ_POLY", 0) == 1;
+    // PKV_MQ_POLY=n (1..3): n of every 8 probability pairs by the FMA-pipe exp2
+    const int poly = env_int("PKV_MQ_POLY", 0);
     if (D == 128) {
-        if (poly)
+        if (poly == 1)
+            k = bf16 ? mq_attention_kernel<128, true, 1> : mq_attention_kernel<128, false, 1>;
+        else if (poly == 2)
+            k = bf16 ? mq_attention_kernel<128, true, 2> : mq_attention_kernel<128, false, 2>;
+        else if (poly == 3)
             k = bf16 ? mq_attention_kernel<128, true, 3> : mq_attention_kernel<128, false, 3>;
         else
             k = bf16 ? mq_attention_kernel<128, true> : mq_attention_kernel<128, false>;

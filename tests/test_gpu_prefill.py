@@ -101,6 +101,16 @@ def test_multi_query_kernel_edge_cases(case):
     gh.assert_close(gh.to_f64(out), ref, case[0], "prefill (multi-query kernel)")
 
 
+@pytest.mark.parametrize("poly", ["1", "2", "3"])
+def test_multi_query_kernel_fma_pipe_exponentials(poly, monkeypatch):
+    # PKV_MQ_POLY=n: n of every 8 probability pairs by the FMA-pipe exp2
+    # (relative error < 8e-6): the same tolerance as the SFU path
+    monkeypatch.setenv("PKV_MQ_POLY", poly)
+    for case in (MQ_CASES[0], MQ_CASES[1]):
+        out, ref, _, _ = _run_case(case, seed=9)
+        gh.assert_close(gh.to_f64(out), ref, case[0], f"prefill, PKV_MQ_POLY={poly}")
+
+
 def test_negative_scale():
     case = (F16, 32, 8, 128, 16, [(600, 200), (50, 1)])
     out, ref, _, _ = _run_case(case, seed=6, scale=-0.07)
