@@ -1009,10 +1009,13 @@ pkv_status pkv_append_decode_attention_shared_prefix(
     float *po = reinterpret_cast<float *>(ws + wl.o);
     float *pm = reinterpret_cast<float *>(ws + wl.m);
     float *pl = reinterpret_cast<float *>(ws + wl.l);
-    cascade_prep_kernel<<<(unsigned)((num_seqs + 7) / 8), 256, (size_t)(num_groups + 1) * 4, (cudaStream_t)stream>>>(
-        group_start, (int)num_groups, shared_lens, context_lens, block_tables, max_blocks_per_seq,
-        (int)k_cache.block_size, (int)num_seqs, g_ref, g_len, shared, suffix, toff, counter, err);
-    if (!cuda_ok(cudaGetLastError()))
+    // a programmatic dependent like the kernels after it (it waits for the
+    // previous kernel before reading anything)
+    if (!cuda_ok(launch_dependent(cascade_prep_kernel, dim3((unsigned)((num_seqs + 7) / 8)), dim3(256),
+                                  (size_t)(num_groups + 1) * 4, (cudaStream_t)stream, group_start, (int)num_groups,
+                                  shared_lens, context_lens, block_tables, max_blocks_per_seq,
+                                  (int)k_cache.block_size, (int)num_seqs, g_ref, g_len, shared, suffix, toff, counter,
+                                  err)))
         return PKV_ERR_CUDA;
     MqArgs a = {};
     a.mode = kMqPrefix;
