@@ -9,23 +9,28 @@
 // everything before it.
 //
 // Kernel design (B200):
-//  * Work unit = (sequence, KV head, block of `tpb` consecutive chunk tokens).
-//    Its rows are the tpb tokens x the G query heads that share the KV head
-//    (tpb * G <= 128): one 128-row tile.  Every K/V tile of the unit's
-//    causal range is loaded once for all of them, so a chunk reads each K/V
-//    position once per row block instead of once per query token.
-//  * S = Q K^T and O += P V are tcgen05.mma (kind::f16, M = 128) with both
-//    operands in shared memory (128-byte swizzled tiles straight from TMA)
-//    and fp32 accumulators in tensor memory: S double-buffered (2 x 128
-//    columns), O in 128 columns.
-//  * Warp roles in a 192-thread CTA: warps 0-3 own one row each (TMEM lane =
-//    row): online softmax of S, P to shared memory, the rare O rescale and
-//    the epilogue; warp 4 is the producer (unit scheduler, TMA loads of Q and
-//    of the K/V tiles through the block table); warp 5 allocates TMEM and one
-//    of its threads issues every MMA.  All hand-offs are mbarriers; every
-//    wait is bounded (time-out -> error word, orderly teardown).
+//  * Work unit = (source, KV head, block of `tpb` consecutive query sources):
+//    a source is a chunk's sequence (its tokens are the queries) or a
+//    sharing group (its members' decode queries over their common prefix).
+//    The rows are the tpb sources x the G query heads that share the KV head
+//    (tpb * G <= 128): one 128-row tile.  Every K/V tile of the unit's range
+//    is loaded once for all of them, so a chunk reads each K/V position once
+//    per row block instead of once per query token.
+//  * S = Q K^T (both operands in shared memory: 128-byte swizzled tiles
+//    straight from TMA) and, per 64-position half h of the tile,
+//    O_h += P_h V_h with P_h read from tensor memory, as tcgen05.mma
+//    (kind::f16, M = 128) with fp32 accumulators in tensor memory: S
+//    double-buffered (2 x 128 columns; P is written over its own scores),
+//    O_0 and O_1 (D columns each).
+//  * Warp roles in a 352-thread CTA: warps 0-7 the softmax (warp w: the rows
+//    of TMEM lane quarter w % 4, the positions of half w / 4 of each tile,
+//    with a running max and sum of its own; the two halves of a row meet in
+//    the epilogue); warp 8 the unit scheduler and the TMA loads of Q and K;
+//    warp 10 the TMA loads of V; warp 9 allocates TMEM and one of its threads
+//    issues every MMA.  All hand-offs are mbarriers; every wait is bounded
+//    (time-out -> error word, orderly teardown).
 //  * Persistent grid (one CTA per SM); units are taken from a global counter
-//    in order of decreasing causal length within each sequence.
+//    in order of decreasing causal length within each source.
 //  * Online softmax in the log2 domain with a lazy rescale: the running
 //    reference max only moves when the tile max exceeds it by more than 2^8,
 //    so P stays <= 256 (exact enough in 16 bits) and O in TMEM is almost
@@ -96,7 +101,7 @@ struct MqSmem {
     // barrier indices
     static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kMqKStages,
                          kVFull = kKEmpty + kMqKStages, kVEmpty = kVFull + kMqVStages, kSFull = kVEmpty + kMqVStages,
-                         kSFree = kSFull + 2, kPFull = kSFree + 2, kODone = kPFull + 2, kUnitFull = kODone + 1,
+                         kPFull = kSFull + 2, kODone = kPFull + 2, kUnitFull = kODone + 1,
                          kUnitEmpty = kUnitFull + 2, kDrain = kUnitEmpty + 2, kXch = kDrain + 1,
                          kNumBars = kXch + 4;
     static constexpr int misc = bars + kNumBars * 8;     // [0..1] unit slots, [2] TMEM base, [3] abort
@@ -247,7 +252,6 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(L::kSFull + i), 1);
-            mbar_init(bar(L::kSFree + i), 1);  // P V of the buffer's last tile is done (its P is read)
             mbar_init(bar(L::kUnitFull + i), 1);
             mbar_init(bar(L::kUnitEmpty + i), 2 + kMqSoftmaxWarps);  // MMA thread, V producer, softmax warps
         }

@@ -94,6 +94,20 @@ def test_named_workload_full_size(name):
               f"max |err| {err:.3e}")
 
 
+def test_long_rows_merged_in_decode(monkeypatch):
+    # rows split over many warps (more than the 16 pieces the whole-group
+    # merge takes): the decode kernel's last piece merges them head by head
+    monkeypatch.setenv("PKV_FOLD_MERGE", "1")
+    spec = custom("long_fold_bf16", 2, 64, 8, 128, 16, BF16, 16, [20000, 12345])
+    w = workloads.make(spec)
+    kc, vc, slots = gh.prepare(w)
+    ref, _, _ = gh.oracle_step(w, kc, vc, slots)
+    for fused in (False, True):
+        step = gh.GpuStep(w, kc, vc, slots)
+        out = step.run_fused(pkv.PKV_PARTITION_AUTO) if fused else step.run(pkv.PKV_PARTITION_AUTO)
+        gh.assert_close(gh.to_f64(out), ref, BF16, f"long rows, merge in decode, fused={fused}")
+
+
 @pytest.mark.parametrize("fold", ["0", "1"], ids=["merge_kernel", "merge_in_decode"])
 def test_split_rows_merged_either_way(small_case, fold, monkeypatch):
     # the work-balanced schedule's split rows, merged by the merge kernel or
