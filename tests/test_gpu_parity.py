@@ -94,6 +94,17 @@ def test_named_workload_full_size(name):
               f"max |err| {err:.3e}")
 
 
+@pytest.mark.parametrize("unit_cost", ["0", "8"])
+def test_balanced_schedule_unit_cost_extremes(small_case, unit_cost, monkeypatch):
+    # the work-balanced order with no virtual tiles per (sequence, head group)
+    # and with the most: ranges that start or end inside the virtual tails
+    monkeypatch.setenv("PKV_UNIT_COST", unit_cost)
+    w, kc, vc, slots, ref, k_ref, v_ref = small_case
+    step = gh.GpuStep(w, kc, vc, slots)
+    out = step.run_fused(pkv.PKV_PARTITION_AUTO)
+    gh.assert_close(gh.to_f64(out), ref, w.spec.dtype, f"{w.spec.name} unit cost {unit_cost}")
+
+
 def test_long_rows_merged_in_decode(monkeypatch):
     # rows split over many warps (more than the 16 pieces the whole-group
     # merge takes): the decode kernel's last piece merges them head by head
