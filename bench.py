@@ -426,8 +426,11 @@ def run_gpu(args, rank, world, local):
         "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
         "roofline": {
             "bound": "hbm",
+            # the split rows are merged by lse_merge_kernel or, where rows
+            # split into few pieces, inside the decode kernel (fold_zero_kernel
+            # then zeroes its counters): the library decides per shape
             "kernel": ("cascade_prep_kernel+mq_attention_kernel+" if cascade else "") + "paged_decode_kernel" +
-                      ("+lse_merge_kernel" if merge_launched else ""),
+                      ("+merge of split rows" if merge_launched else ""),
             "achieved": round(achieved, 2),
             "peak": peaks["hbm_gbs"],
             "peak_source": peaks["source"],
@@ -435,7 +438,8 @@ def run_gpu(args, rank, world, local):
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             # shared-prefix blocks counted once: the bandwidth really needed
             "frac_unique": round(nb_bytes["unique_total"] / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "traffic": profiled_traffic(sp.name),
+            # the committed profile covers the plain decode step only
+            "traffic": None if cascade else profiled_traffic(sp.name),
             "algorithmic_bytes_per_launch": nb_bytes["total"],
             "us_per_launch": round(dec_ms * 1e3, 3),
         },
