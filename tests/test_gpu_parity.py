@@ -76,7 +76,7 @@ FULL_MODES = {
 def test_named_workload_full_size(name):
     w = workloads.make(name)
     kc, vc, slots = gh.prepare(w)
-    pairs = None if name == "tiny" else gh.sample_pairs(w, 64)
+    pairs = None if name == "tiny" else gh.sample_pairs(w, 256)
     ref, k_ref, v_ref = gh.oracle_step(w, kc, vc, slots, pairs=pairs)
     step = gh.GpuStep(w, kc, vc, slots)
     for mode, fused in [(m, f) for m in FULL_MODES[name] for f in (False, True)]:

@@ -78,6 +78,22 @@ def test_shared_prefix_matches_oracle(spec, append):
     gh.assert_close(gh.to_f64(step.out), ref, spec.dtype, f"shared prefix {spec.name}")
 
 
+def test_continuous_batching_step_full_size():
+    # the continuous-batching workload at full size (256 sequences, groups of
+    # 16 sharing a 2048-token prefix) through the shared-prefix call, as the
+    # benchmark runs it: pools bit for bit, 256 sampled (sequence, head) rows
+    w = workloads.make("cb_mixed")
+    kc, vc, slots = gh.prepare(w)
+    pairs = gh.sample_pairs(w, 256)
+    ref, k_ref, v_ref = gh.oracle_step(w, kc, vc, slots, pairs=pairs)
+    starts, claims = _groups_of(w)
+    step = _run(w, kc, vc, slots, starts, claims, append=True)
+    assert np.array_equal(gh.host_bits(step.kc), k_ref) and np.array_equal(gh.host_bits(step.vc), v_ref)
+    got = gh.to_f64(step.out)
+    assert np.all(np.isfinite(got))
+    gh.assert_close(got[pairs[:, 0], pairs[:, 1]], ref, w.spec.dtype, "cb_mixed, shared-prefix call")
+
+
 def test_groups_from_the_allocator():
     spec = SPECS[0]
     w = workloads.make(spec)
